@@ -1,0 +1,135 @@
+/*
+ * lard.h -- C ABI of liblard: the linear-memory relation-KL kernel of
+ * LinearARD (relation distillation for RoPE-scaled students), for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Method, as defined on the pages this library follows:
+ *   "LinearARD: Linear-Memory Attention Distillation for RoPE Restoration"
+ *   (papernotes.org notes), 方法详解 / 关键设计 1: for a head, teacher (m = t)
+ *   and student (m = s) projections X_m, Y_m in R^{n x d} give relation
+ *   logits Z_m = tau * X_m Y_m^T under a causal mask M; R_m is their
+ *   row-wise softmax; the loss is the row-averaged forward KL(R_t || R_s),
+ *   summed over the Q/Q, K/K and V/V relations (lambda = 1, section
+ *   损失函数 / 训练策略).
+ *   Same page, 关键设计 3: Phase 1 streams tiles and keeps only the per-row
+ *   statistic LSE_m(i) = log sum_k exp Z_m(i,k) in HBM (O(BHn) memory);
+ *   Phase 2 recomputes 128 x 128 tiles of Z_s and Z_t on chip, rebuilds
+ *   R = exp(Z - LSE), forms dZ = (R_s - R_t)/n and contracts it with the
+ *   projections into dX_s and dY_s, never storing an n x n map.
+ *   LinearARD abstract (fugumt.com page): the kernel computes the exact KL
+ *   divergence and gradients from per-token log-sum-exp statistics.
+ *
+ * Readings this library takes where the pages are silent:
+ *   - tau is a parameter (1/sqrt(d) in the usual setting), tau > 0;
+ *   - the causal mask keeps j <= i (diagonal included); causal = 0 gives the
+ *     plain full-row softmax;
+ *   - the loss of one (batch, head) is (1/n) sum_i KL_i; heads and batch
+ *     entries are summed; a caller sums the three relations;
+ *   - gradients carry the chain-rule factor tau of Z = tau X Y^T:
+ *     dX_s = tau dZ Y_s, dY_s = tau dZ^T X_s; the teacher gets none;
+ *   - for a self-relation (Y = X) the caller adds the two partials.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major [B, H, n, d], contiguous, in device memory of
+ *     the GPU that runs the call, base addresses 16-byte aligned.  Inputs
+ *     are bf16 (LARD_DTYPE_BF16) or fp32 (LARD_DTYPE_FP32); every output is
+ *     fp32.  The caller allocates and owns every buffer; the library
+ *     allocates no device memory.
+ *   - Work is enqueued asynchronously on `stream` (0 = legacy default
+ *     stream); results are valid once the stream reaches that point.
+ *   - Argument errors are reported synchronously, before anything is
+ *     enqueued, and nothing is written.  Launch errors map to LARD_ERR_CUDA.
+ *   - Every wait inside the kernels has a time limit; a wait that runs out
+ *     makes the kernel stop early and sets a device-side fault word that
+ *     lard_device_status() reports as LARD_ERR_TIMEOUT.
+ *   - Supported: d in {64, 128} for bf16, d a multiple of 32 up to 256 for
+ *     fp32; any n >= 1 (ragged last tile handled); B*H*n*d < 2^40.
+ *   - Calls are thread-safe.  Inputs may alias each other (Y = X).
+ */
+#ifndef LARD_H
+#define LARD_H
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define LARD_API __attribute__((visibility("default")))
+#else
+#define LARD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LARD_OK = 0,
+    LARD_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, non-finite scalar, aliasing */
+    LARD_ERR_UNSUPPORTED = 2, /* head dim or dtype not built, or a GPU other than sm_100 */
+    LARD_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+    LARD_ERR_TIMEOUT = 4      /* a kernel wait ran out of time (see lard_device_status) */
+} lard_status;
+
+typedef enum { LARD_DTYPE_BF16 = 0, LARD_DTYPE_FP32 = 1 } lard_dtype;
+
+/*
+ * Phase 1 (LinearARD notes, 关键设计 3, first phase): per-row log-sum-exp of
+ * the teacher and student relation logits and the row KL, streamed over
+ * 128 x 128 tiles without materialising Z.
+ *
+ *   Xt, Yt, Xs, Ys  inputs [B, H, n, d] (teacher X, teacher Y, student X,
+ *                   student Y).  Yt may equal Xt and Ys may equal Xs.
+ *   tau             logit scale, finite and > 0.
+ *   causal          1: mask j > i; 0: no mask.
+ *   lse_t, lse_s    out [B, H, n]: LSE_m(i) = log sum_{j allowed} exp Z_m(i,j).
+ *   row_kl          out [B, H, n]: KL(R_t(i,.) || R_s(i,.)).
+ *   loss_bh         out [B*H] or NULL: (1/n) sum_i row_kl.
+ *   loss_total      out [1] or NULL: sum of loss_bh (requires loss_bh).
+ * Extra device memory beyond the caller's buffers: none.  The HBM state
+ * kept between the phases is lse_t and lse_s, 8 bytes per row.
+ */
+LARD_API lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys,
+                        lard_dtype dtype, int B, int H, int n, int d, float tau, int causal,
+                        float* lse_t, float* lse_s, float* row_kl,
+                        float* loss_bh, float* loss_total, cudaStream_t stream);
+
+/*
+ * Phase 2 (LinearARD notes, 关键设计 3, second phase): recompute Z_t and Z_s
+ * tile by tile, rebuild R from the Phase-1 LSEs, form dZ = (R_s - R_t)/n and
+ * contract it into the student gradients.
+ *
+ *   Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal: as for lard_kl_fwd
+ *                   (must be the same values that produced lse_t / lse_s).
+ *   lse_t, lse_s    in [B, H, n], written by lard_kl_fwd.
+ *   grad_scale      g, finite: upstream gradient of the summed loss.
+ *   dXs, dYs        out [B, H, n, d] fp32, overwritten:
+ *                   dXs = g * dL/dXs = g * tau * dZ Y_s,
+ *                   dYs = g * dL/dYs = g * tau * dZ^T X_s,
+ *                   with L = sum over (b, h) of the row-averaged KL.
+ *                   They must not overlap each other or any input.
+ * The bf16 path accumulates dXs with fp32 atomic adds, so its last bits
+ * depend on the order in which tiles finish; the fp32 path is deterministic.
+ */
+LARD_API lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys,
+                        lard_dtype dtype, int B, int H, int n, int d, float tau, int causal,
+                        const float* lse_t, const float* lse_s, float grad_scale,
+                        float* dXs, float* dYs, cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+LARD_API const char* lard_status_string(lard_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side fault word of
+ * the current device.  Returns LARD_ERR_TIMEOUT if a kernel wait ran out of
+ * time since the last check (and stores the fault bits in *fault_bits if it
+ * is not NULL), LARD_ERR_CUDA if synchronisation failed, else LARD_OK.
+ */
+LARD_API lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+LARD_API int lard_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LARD_H */

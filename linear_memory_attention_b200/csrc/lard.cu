@@ -1,0 +1,334 @@
+// lard.cu -- the C ABI of liblard (declared in include/lard.h): argument
+// checks, per-device setup, TMA tensor maps and kernel launches.  Every step
+// of the relation-KL computation runs in the kernels of the included headers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "lard.h"
+#include "lard_kernel_common.cuh"
+#include "lard_bwd_tc.cuh"
+#include "lard_fp32.cuh"
+#include "lard_fwd_tc.cuh"
+
+namespace {
+
+constexpr int kVersion = 100;                          // 0.1.0
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxDevices = 64;
+constexpr long long kMaxElems = 1LL << 40;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+bool g_ready[kMaxDevices];
+lard_status g_dev_status[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+// Restores the caller's current device when a call returns.
+struct DeviceGuard {
+    int prev = -1;
+    DeviceGuard() {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            prev = -1;
+            cudaGetLastError();
+        }
+    }
+    ~DeviceGuard() {
+        if (prev >= 0) cudaSetDevice(prev);
+    }
+};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+bool d_supported(lard_dtype dt, int d) {
+    if (dt == LARD_DTYPE_BF16) return d == 64 || d == 128;
+    return d >= 32 && d <= 256 && d % 32 == 0;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// One-time setup of device `dev` (made current by the caller).
+lard_status setup_device(int dev) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev < 0 || dev >= kMaxDevices) return LARD_ERR_UNSUPPORTED;
+    if (g_ready[dev]) return g_dev_status[dev];
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return LARD_ERR_CUDA;
+    lard_status st = LARD_OK;
+    if (major != 10 || minor != 0) st = LARD_ERR_UNSUPPORTED;  // built for sm_100a only
+    if (st == LARD_OK && !g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                             &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            st = LARD_ERR_CUDA;
+        else
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (st == LARD_OK) {
+        bool ok = set_smem(lard::lard_fwd_tc_kernel<64>, lard::FwdLayout<64>::SMEM_BYTES) == cudaSuccess &&
+                  set_smem(lard::lard_fwd_tc_kernel<128>, lard::FwdLayout<128>::SMEM_BYTES) == cudaSuccess &&
+                  set_smem(lard::lard_bwd_tc_kernel<64>, lard::BwdLayout<64>::SMEM_BYTES) == cudaSuccess &&
+                  set_smem(lard::lard_bwd_tc_kernel<128>, lard::BwdLayout<128>::SMEM_BYTES) == cudaSuccess;
+        if (!ok) st = LARD_ERR_CUDA;
+    }
+    g_dev_status[dev] = st;
+    g_ready[dev] = true;
+    return st;
+}
+
+// Finds the GPU that holds `ptr`, makes it current and sets it up.
+lard_status select_device(const void* ptr) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return LARD_ERR_INVALID_ARG;
+    }
+    if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) return LARD_ERR_INVALID_ARG;
+    if (cudaSetDevice(at.device) != cudaSuccess) return LARD_ERR_CUDA;
+    return setup_device(at.device);
+}
+
+// 3-D tensor map over [BH, n, d] bf16 with 64 x 128 boxes, 128-byte swizzle.
+// Rows past n read as zeros.
+bool make_map(CUtensorMap* m, const void* base, long long BH, int n, int d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n) * d * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Checks shared by both phases.
+lard_status check_common(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
+                         int B, int H, int n, int d, float tau, int causal, long long* BH_out) {
+    if (!Xt || !Yt || !Xs || !Ys) return LARD_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || n < 1 || d < 1) return LARD_ERR_INVALID_ARG;
+    if (!(std::isfinite(tau) && tau > 0.f)) return LARD_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return LARD_ERR_INVALID_ARG;
+    if (dtype != LARD_DTYPE_BF16 && dtype != LARD_DTYPE_FP32) return LARD_ERR_UNSUPPORTED;
+    if (!d_supported(dtype, d)) return LARD_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    if (BH > INT_MAX / 2 || BH * n > kMaxElems / d) return LARD_ERR_INVALID_ARG;
+    const long long T = (n + 127) / 128;
+    if (BH * T > INT_MAX) return LARD_ERR_INVALID_ARG;
+    for (const void* p : {Xt, Yt, Xs, Ys})
+        if (!aligned(p, 16)) return LARD_ERR_INVALID_ARG;
+    *BH_out = BH;
+    return LARD_OK;
+}
+
+size_t in_bytes(lard_dtype dt, long long BH, int n, int d) {
+    return static_cast<size_t>(BH) * n * d * (dt == LARD_DTYPE_BF16 ? 2 : 4);
+}
+
+template <int E>
+void launch_fwd_fp32(const float* Xt, const float* Yt, const float* Xs, const float* Ys,
+                     const lard::Fp32Params& p, float* lse_t, float* lse_s, float* row_kl, cudaStream_t s) {
+    const long long warps = static_cast<long long>(p.BH) * p.n;
+    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+    lard::lard_fwd_fp32_kernel<E><<<blocks, 256, 0, s>>>(Xt, Yt, Xs, Ys, p, lse_t, lse_s, row_kl);
+}
+
+template <int E>
+void launch_bwd_fp32(const float* Xt, const float* Yt, const float* Xs, const float* Ys,
+                     const lard::Fp32Params& p, const float* lse_t, const float* lse_s, float* dXs,
+                     float* dYs, cudaStream_t s) {
+    const long long warps = static_cast<long long>(p.BH) * p.n;
+    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+    lard::lard_bwd_rownorm_fp32_kernel<E><<<blocks, 256, 0, s>>>(Xt, Yt, Xs, Ys, p, lse_t, lse_s, dXs);
+    lard::lard_bwd_dy_fp32_kernel<E><<<blocks, 256, 0, s>>>(Xt, Yt, Xs, Ys, p, lse_t, lse_s, dXs, dYs);
+    lard::lard_bwd_dx_fp32_kernel<E><<<blocks, 256, 0, s>>>(Xt, Yt, Xs, Ys, p, lse_t, lse_s, dXs);
+}
+
+#define LARD_DISPATCH_E(d, F, ...)                   \
+    switch ((d) / 32) {                              \
+        case 1: F<1>(__VA_ARGS__); break;            \
+        case 2: F<2>(__VA_ARGS__); break;            \
+        case 3: F<3>(__VA_ARGS__); break;            \
+        case 4: F<4>(__VA_ARGS__); break;            \
+        case 5: F<5>(__VA_ARGS__); break;            \
+        case 6: F<6>(__VA_ARGS__); break;            \
+        case 7: F<7>(__VA_ARGS__); break;            \
+        default: F<8>(__VA_ARGS__); break;           \
+    }
+
+}  // namespace
+
+extern "C" {
+
+lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
+                        int B, int H, int n, int d, float tau, int causal, float* lse_t, float* lse_s,
+                        float* row_kl, float* loss_bh, float* loss_total, cudaStream_t stream) {
+    long long BH = 0;
+    lard_status st = check_common(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, &BH);
+    if (st != LARD_OK) return st;
+    if (!lse_t || !lse_s || !row_kl) return LARD_ERR_INVALID_ARG;
+    if (loss_total && !loss_bh) return LARD_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)lse_t, (const void*)lse_s, (const void*)row_kl, (const void*)loss_bh,
+                          (const void*)loss_total})
+        if (p && !aligned(p, 4)) return LARD_ERR_INVALID_ARG;
+    const size_t nin = in_bytes(dtype, BH, n, d), nrow = static_cast<size_t>(BH) * n * 4;
+    const void* outs[5] = {lse_t, lse_s, row_kl, loss_bh, loss_total};
+    const size_t outn[5] = {nrow, nrow, nrow, static_cast<size_t>(BH) * 4, 4};
+    for (int a = 0; a < 5; ++a) {
+        if (!outs[a]) continue;
+        for (const void* in : {Xt, Yt, Xs, Ys})
+            if (overlap(outs[a], outn[a], in, nin)) return LARD_ERR_INVALID_ARG;
+        for (int b = a + 1; b < 5; ++b)
+            if (outs[b] && overlap(outs[a], outn[a], outs[b], outn[b])) return LARD_ERR_INVALID_ARG;
+    }
+
+    DeviceGuard guard;
+    st = select_device(Xt);
+    if (st != LARD_OK) return st;
+
+    const int T = (n + 127) / 128;
+    if (dtype == LARD_DTYPE_BF16) {
+        CUtensorMap mxt, myt, mxs, mys;
+        if (!make_map(&mxt, Xt, BH, n, d) || !make_map(&myt, Yt, BH, n, d) || !make_map(&mxs, Xs, BH, n, d) ||
+            !make_map(&mys, Ys, BH, n, d))
+            return LARD_ERR_INVALID_ARG;
+        lard::TcFwdParams p;
+        p.BH = static_cast<int>(BH);
+        p.n = n;
+        p.T = T;
+        p.causal = causal;
+        p.tau = tau;
+        p.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
+        p.lse_t = lse_t;
+        p.lse_s = lse_s;
+        p.row_kl = row_kl;
+        p.wait_ns = kWaitLimitNs;
+        const unsigned grid = static_cast<unsigned>(BH * T);
+        if (d == 128)
+            lard::lard_fwd_tc_kernel<128><<<grid, 384, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+        else
+            lard::lard_fwd_tc_kernel<64><<<grid, 384, lard::FwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+    } else {
+        lard::Fp32Params p;
+        p.BH = static_cast<int>(BH);
+        p.n = n;
+        p.causal = causal;
+        p.tau = tau;
+        p.dz_scale = 0.0;
+        LARD_DISPATCH_E(d, launch_fwd_fp32, static_cast<const float*>(Xt), static_cast<const float*>(Yt),
+                        static_cast<const float*>(Xs), static_cast<const float*>(Ys), p, lse_t, lse_s, row_kl,
+                        stream);
+    }
+    if (loss_bh) lard::lard_loss_rows_kernel<<<static_cast<unsigned>(BH), 256, 0, stream>>>(row_kl, n, loss_bh);
+    if (loss_total) lard::lard_loss_total_kernel<<<1, 256, 0, stream>>>(loss_bh, static_cast<int>(BH), loss_total);
+    return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
+}
+
+lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
+                        int B, int H, int n, int d, float tau, int causal, const float* lse_t,
+                        const float* lse_s, float grad_scale, float* dXs, float* dYs, cudaStream_t stream) {
+    long long BH = 0;
+    lard_status st = check_common(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, &BH);
+    if (st != LARD_OK) return st;
+    if (!lse_t || !lse_s || !dXs || !dYs) return LARD_ERR_INVALID_ARG;
+    if (!std::isfinite(grad_scale)) return LARD_ERR_INVALID_ARG;
+    if (!aligned(lse_t, 4) || !aligned(lse_s, 4) || !aligned(dXs, 16) || !aligned(dYs, 16))
+        return LARD_ERR_INVALID_ARG;
+    const size_t nin = in_bytes(dtype, BH, n, d), ngrad = static_cast<size_t>(BH) * n * d * 4;
+    const size_t nrow = static_cast<size_t>(BH) * n * 4;
+    if (overlap(dXs, ngrad, dYs, ngrad)) return LARD_ERR_INVALID_ARG;
+    for (const void* g : {(const void*)dXs, (const void*)dYs}) {
+        for (const void* in : {Xt, Yt, Xs, Ys})
+            if (overlap(g, ngrad, in, nin)) return LARD_ERR_INVALID_ARG;
+        if (overlap(g, ngrad, lse_t, nrow) || overlap(g, ngrad, lse_s, nrow)) return LARD_ERR_INVALID_ARG;
+    }
+
+    DeviceGuard guard;
+    st = select_device(Xt);
+    if (st != LARD_OK) return st;
+
+    const int T = (n + 127) / 128;
+    const double dz_scale = static_cast<double>(tau) * grad_scale / n;
+    if (dtype == LARD_DTYPE_BF16) {
+        CUtensorMap mxt, myt, mxs, mys;
+        if (!make_map(&mxt, Xt, BH, n, d) || !make_map(&myt, Yt, BH, n, d) || !make_map(&mxs, Xs, BH, n, d) ||
+            !make_map(&mys, Ys, BH, n, d))
+            return LARD_ERR_INVALID_ARG;
+        if (cudaMemsetAsync(dXs, 0, ngrad, stream) != cudaSuccess) return LARD_ERR_CUDA;
+        lard::TcBwdParams p;
+        p.BH = static_cast<int>(BH);
+        p.n = n;
+        p.T = T;
+        p.causal = causal;
+        p.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
+        p.dz_scale = static_cast<float>(dz_scale);
+        p.lse_t = lse_t;
+        p.lse_s = lse_s;
+        p.dXs = dXs;
+        p.dYs = dYs;
+        p.wait_ns = kWaitLimitNs;
+        const unsigned grid = static_cast<unsigned>(BH * T);
+        if (d == 128)
+            lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+        else
+            lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+    } else {
+        lard::Fp32Params p;
+        p.BH = static_cast<int>(BH);
+        p.n = n;
+        p.causal = causal;
+        p.tau = tau;
+        p.dz_scale = dz_scale;
+        LARD_DISPATCH_E(d, launch_bwd_fp32, static_cast<const float*>(Xt), static_cast<const float*>(Yt),
+                        static_cast<const float*>(Xs), static_cast<const float*>(Ys), p, lse_t, lse_s, dXs, dYs,
+                        stream);
+    }
+    return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
+}
+
+const char* lard_status_string(lard_status s) {
+    switch (s) {
+        case LARD_OK: return "LARD_OK";
+        case LARD_ERR_INVALID_ARG: return "LARD_ERR_INVALID_ARG";
+        case LARD_ERR_UNSUPPORTED: return "LARD_ERR_UNSUPPORTED";
+        case LARD_ERR_CUDA: return "LARD_ERR_CUDA";
+        case LARD_ERR_TIMEOUT: return "LARD_ERR_TIMEOUT";
+    }
+    return "LARD_ERR_UNKNOWN";
+}
+
+lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LARD_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, lard::g_lard_fault, sizeof(v)) != cudaSuccess) return LARD_ERR_CUDA;
+    if (fault_bits) *fault_bits = v;
+    if (v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(lard::g_lard_fault, &zero, sizeof(zero)) != cudaSuccess) return LARD_ERR_CUDA;
+        return LARD_ERR_TIMEOUT;
+    }
+    return LARD_OK;
+}
+
+int lard_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,354 @@
+// lard_bwd_tc.cuh -- Phase 2 on the 5th-generation tensor cores (bf16 inputs).
+//
+// LinearARD notes (papernotes.org), 关键设计 3, second phase: per T_r x T_c =
+// 128 x 128 tile, recompute the student and teacher logits on chip, rebuild
+// R = exp(Z - LSE) from the Phase-1 statistics, form dZ = (R_s - R_t)/n and
+// contract it with the projections into dX_s and dY_s.  Fully masked tiles
+// (J > I) are never visited.
+//
+// One CTA owns a 128-column block J of one (batch, head); its dY_s[J]
+// accumulator stays in TMEM for the whole sweep over the row blocks I >= J
+// (all I without the mask), and each tile's dX_s[I] contribution is added
+// to HBM with fp32 vector atomics.
+// TMEM (512 columns): dY [0, D), S_t [128, 256), S_s [256, 384), dX [384, 384 + D).
+// Shared memory: Y_t[J], Y_s[J] resident; a 2-stage ring of (X_t[I], X_s[I]);
+// one 128 x 128 bf16 dZ tile, 128B-swizzled, read by both gradient GEMMs:
+//   GEMM 3  dY[J] += dZ^T X_s[I]   (A = dZ as MN-major, B = X_s as MN-major)
+//   GEMM 4  dX[I]  = dZ  Y_s[J]    (A = dZ as K-major,  B = Y_s as MN-major)
+// Roles (512 threads):
+//   warp 0       TMA producer          warp 1   TMEM owner, MMA issuer
+//   warps 4-11   dZ: one row per thread, one 64-column half per warpgroup
+//   warps 12-15  dX drain (TMEM -> red.global.add) and the final dY store
+#pragma once
+
+#include "lard_kernel_common.cuh"
+
+namespace lard {
+
+struct TcBwdParams {
+    int BH, n, T, causal;
+    float cfac;      // tau * log2(e)
+    float dz_scale;  // tau * grad_scale / n: dZ and the chain-rule tau in one factor
+    const float* lse_t;
+    const float* lse_s;
+    float* dXs;
+    float* dYs;
+    unsigned long long wait_ns;
+};
+
+template <int D>
+struct BwdLayout {
+    static constexpr int KC = D / 64;
+    static constexpr int TILE = KC * 16384;
+    static constexpr int NS = 2;
+    static constexpr int OFF_YT = 0;
+    static constexpr int OFF_YS = TILE;
+    static constexpr int OFF_X = 2 * TILE;  // stage s: X_t at OFF_X + 2*s*TILE, X_s after it
+    static constexpr int OFF_DZ = OFF_X + NS * 2 * TILE;
+    static constexpr int OFF_CTRL = OFF_DZ + 32768;
+    static constexpr int CTRL_BYTES = 1024;
+    static constexpr int SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;
+};
+
+struct BwdCtrl {
+    uint64_t y_full;
+    uint64_t x_full[2];
+    uint64_t x_empty[2];
+    uint64_t s_full, s_free, dz_full, dz_free, dx_full, dx_free, dy_full, mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+static_assert(sizeof(BwdCtrl) <= 1024, "control block too large");
+
+constexpr uint32_t kTmemDY = 0, kTmemSt = 128, kTmemSs = 256, kTmemDX = 384;
+
+template <int D>
+__global__ void __launch_bounds__(512, 1)
+    lard_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_xt,
+                       const __grid_constant__ CUtensorMap tm_yt,
+                       const __grid_constant__ CUtensorMap tm_xs,
+                       const __grid_constant__ CUtensorMap tm_ys, const TcBwdParams p) {
+    using L = BwdLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
+    BwdCtrl* ctrl = reinterpret_cast<BwdCtrl*>(smem + L::OFF_CTRL);
+    volatile int* abort_flag = &ctrl->abort_flag;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // Head-major order, longest column blocks first within a head: the blocks
+    // resident at any time then share one head's X tiles and dX rows in L2.
+    const int bh = static_cast<int>(blockIdx.x) / p.T;
+    const int J = static_cast<int>(blockIdx.x) % p.T;
+    const int K = p.causal ? (p.T - J) : p.T;
+    auto row_block = [&](int k) { return p.causal ? (J + k) : k; };
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&ctrl->y_full, 1);
+        for (int s = 0; s < L::NS; ++s) {
+            ptx::mbar_init(&ctrl->x_full[s], 1);
+            ptx::mbar_init(&ctrl->x_empty[s], 1);
+        }
+        ptx::mbar_init(&ctrl->s_full, 1);
+        ptx::mbar_init(&ctrl->s_free, 8);
+        ptx::mbar_init(&ctrl->dz_full, 8);
+        ptx::mbar_init(&ctrl->dz_free, 1);
+        ptx::mbar_init(&ctrl->dx_full, 1);
+        ptx::mbar_init(&ctrl->dx_free, 4);
+        ptx::mbar_init(&ctrl->dy_full, 1);
+        ptx::mbar_init(&ctrl->mma_done, 1);
+        ctrl->abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tensormap(&tm_xt);
+        ptx::prefetch_tensormap(&tm_yt);
+        ptx::prefetch_tensormap(&tm_xs);
+        ptx::prefetch_tensormap(&tm_ys);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&ctrl->tmem_base, 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = ctrl->tmem_base;
+    const uint64_t lim = p.wait_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            ptx::mbar_arrive_expect_tx(&ctrl->y_full, 2 * L::TILE);
+            for (int c = 0; c < L::KC; ++c) {
+                ptx::tma_load_3d(smem + L::OFF_YT + c * 16384, &tm_yt, &ctrl->y_full, c * 64, J * 128, bh);
+                ptx::tma_load_3d(smem + L::OFF_YS + c * 16384, &tm_ys, &ctrl->y_full, c * 64, J * 128, bh);
+            }
+        }
+        __syncwarp();
+        int issued = 0;
+        for (int k = 0; k < K; ++k) {
+            const int s = k & 1, rnd = k >> 1;
+            bool ok = ptx::mbar_wait(&ctrl->x_empty[s], (rnd & 1) ^ 1, abort_flag, lim, &g_lard_fault,
+                                     kFaultBwdProducer);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (lane == 0) {
+                const int I = row_block(k);
+                uint8_t* xt = smem + L::OFF_X + 2 * s * L::TILE;
+                ptx::mbar_arrive_expect_tx(&ctrl->x_full[s], 2 * L::TILE);
+                for (int c = 0; c < L::KC; ++c) {
+                    ptx::tma_load_3d(xt + c * 16384, &tm_xt, &ctrl->x_full[s], c * 64, I * 128, bh);
+                    ptx::tma_load_3d(xt + L::TILE + c * 16384, &tm_xs, &ctrl->x_full[s], c * 64, I * 128, bh);
+                }
+            }
+            __syncwarp();
+            ++issued;
+        }
+        ptx::mbar_drain(&ctrl->y_full, 0, lim);
+        for (int s = 0; s < L::NS && s < issued; ++s) {
+            const int last = s + L::NS * ((issued - 1 - s) / L::NS);
+            ptx::mbar_drain(&ctrl->x_full[s], (last / L::NS) & 1, lim);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t kIdescS = ptx::idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t kIdescDY = ptx::idesc_bf16(128, D, 1, 1);
+        constexpr uint32_t kIdescDX = ptx::idesc_bf16(128, D, 0, 1);
+        const uint32_t syt = ptx::smem_u32(smem + L::OFF_YT);
+        const uint32_t sys = ptx::smem_u32(smem + L::OFF_YS);
+        const uint32_t sdz = ptx::smem_u32(smem + L::OFF_DZ);
+        auto issue_s = [&](int k) {
+            const uint32_t sxt = ptx::smem_u32(smem + L::OFF_X + 2 * (k & 1) * L::TILE);
+            const uint32_t sxs = sxt + L::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                ptx::umma_bf16(tmem + kTmemSt, ptx::sdesc_sw128(sxt + koff, 16, 1024),
+                               ptx::sdesc_sw128(syt + koff, 16, 1024), kIdescS, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                ptx::umma_bf16(tmem + kTmemSs, ptx::sdesc_sw128(sxs + koff, 16, 1024),
+                               ptx::sdesc_sw128(sys + koff, 16, 1024), kIdescS, kk > 0);
+            }
+            ptx::umma_commit(&ctrl->s_full);
+        };
+        bool ok = ptx::mbar_wait(&ctrl->y_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma) &&
+                  ptx::mbar_wait(&ctrl->x_full[0], 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            ptx::tc_fence_after();
+            if (lane == 0) issue_s(0);
+            __syncwarp();
+        }
+        for (int k = 0; ok && k < K; ++k) {
+            if (k + 1 < K) {
+                ok = ptx::mbar_wait(&ctrl->x_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag, lim,
+                                    &g_lard_fault, kFaultBwdMma) &&
+                     ptx::mbar_wait(&ctrl->s_free, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                ptx::tc_fence_after();
+                if (lane == 0) issue_s(k + 1);
+                __syncwarp();
+            }
+            ok = ptx::mbar_wait(&ctrl->dz_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma) &&
+                 ptx::mbar_wait(&ctrl->dx_free, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            ptx::tc_fence_after();
+            if (lane == 0) {
+                const uint32_t sxs = ptx::smem_u32(smem + L::OFF_X + 2 * (k & 1) * L::TILE) + L::TILE;
+                // GEMM 3: dY[J] (+)= dZ^T X_s[I]; K runs over the 128 rows i, 16 per step.
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::umma_bf16(tmem + kTmemDY, ptx::sdesc_sw128(sdz + kk * 2048, 16384, 1024),
+                                   ptx::sdesc_sw128(sxs + kk * 2048, 16384, 1024), kIdescDY,
+                                   (k > 0 || kk > 0) ? 1u : 0u);
+                // GEMM 4: dX[I] = dZ Y_s[J]; K runs over the 128 columns j.
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::umma_bf16(tmem + kTmemDX,
+                                   ptx::sdesc_sw128(sdz + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                   ptx::sdesc_sw128(sys + kk * 2048, 16384, 1024), kIdescDX,
+                                   kk > 0 ? 1u : 0u);
+                ptx::umma_commit(&ctrl->dz_free);
+                ptx::umma_commit(&ctrl->x_empty[k & 1]);
+                ptx::umma_commit(&ctrl->dx_full);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            if (ok) ptx::umma_commit(&ctrl->dy_full);
+            ptx::umma_commit(&ctrl->mma_done);
+        }
+        __syncwarp();
+        ptx::mbar_drain(&ctrl->mma_done, 0, lim);
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------ dZ
+        const int q = warp & 3;
+        const int hcol = (warp - 4) >> 2;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t sdz_row = ptx::smem_u32(smem + L::OFF_DZ) + hcol * 16384 + r * 128;
+        const float cf = p.cfac;
+        const float dzs = p.dz_scale;
+        const float kLog2e = 1.4426950408889634f;
+        // The row's LSEs for tile k are loaded one tile ahead, off the critical path.
+        auto load_lse = [&](int k, float& t, float& s) {
+            const int i = row_block(k) * 128 + r;
+            const size_t o = static_cast<size_t>(bh) * p.n + (i < p.n ? i : 0);
+            t = p.lse_t[o];
+            s = p.lse_s[o];
+        };
+        float nlt = 0.f, nls = 0.f;
+        load_lse(0, nlt, nls);
+        for (int k = 0; k < K; ++k) {
+            const int I = row_block(k);
+            const int i = I * 128 + r;
+            const bool row_ok = i < p.n;
+            const float bt = row_ok ? nlt * kLog2e : 0.f;
+            const float bs = row_ok ? nls * kLog2e : 0.f;
+            if (k + 1 < K) load_lse(k + 1, nlt, nls);
+            int jlim = 128;
+            if (!row_ok) jlim = 0;
+            else if (p.causal) { if (I == J) jlim = r + 1; }
+            else if (J == p.T - 1) jlim = p.n - J * 128;
+
+            bool ok = ptx::mbar_wait(&ctrl->s_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdSoftmax);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            ptx::tc_fence_after();
+            uint32_t pk[32];
+#pragma unroll
+            for (int round = 0; round < 2; ++round) {
+                const int cb = hcol * 64 + round * 32;
+                float st[32], ss[32];
+                __syncwarp();
+                ptx::tmem_ld32(lane_base + kTmemSt + cb, st);
+                ptx::tmem_ld32(lane_base + kTmemSs + cb, ss);
+                ptx::tmem_ld_wait(st);
+                ptx::reg_dep(ss);
+                if (round == 1) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&ctrl->s_free);
+                }
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const float rt0 = ptx::ex2(fmaf(st[c], cf, -bt));
+                    const float rs0 = ptx::ex2(fmaf(ss[c], cf, -bs));
+                    const float rt1 = ptx::ex2(fmaf(st[c + 1], cf, -bt));
+                    const float rs1 = ptx::ex2(fmaf(ss[c + 1], cf, -bs));
+                    const float d0 = (cb + c < jlim) ? (rs0 - rt0) * dzs : 0.f;
+                    const float d1 = (cb + c + 1 < jlim) ? (rs1 - rt1) * dzs : 0.f;
+                    pk[round * 16 + (c >> 1)] = ptx::pack_bf16x2(d0, d1);
+                }
+            }
+            ok = ptx::mbar_wait(&ctrl->dz_free, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault, kFaultBwdSoftmax);
+            if (!__all_sync(0xffffffffu, ok)) break;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                ptx::st_shared_v4(sdz_row + ((u ^ (r & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                                  pk[4 * u + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ctrl->dz_full);
+        }
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ dX drain, dY store
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        bool ok = true;
+        for (int k = 0; k < K; ++k) {
+            const int i = row_block(k) * 128 + r;
+            ok = ptx::mbar_wait(&ctrl->dx_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            ptx::tc_fence_after();
+            float* dst = p.dXs + (static_cast<size_t>(bh) * p.n + (i < p.n ? i : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                __syncwarp();
+                ptx::tmem_ld32(lane_base + kTmemDX + c * 32, v);
+                ptx::tmem_ld_wait(v);
+                if (i < p.n) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        ptx::red_add_v4(dst + c * 32 + 4 * u, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ctrl->dx_free);
+        }
+        if (ok) {
+            ok = ptx::mbar_wait(&ctrl->dy_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdEpilogue);
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (ok) {
+            ptx::tc_fence_after();
+            const int j = J * 128 + r;
+            float* dst = p.dYs + (static_cast<size_t>(bh) * p.n + (j < p.n ? j : 0)) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                __syncwarp();
+                ptx::tmem_ld32(lane_base + kTmemDY + c * 32, v);
+                ptx::tmem_ld_wait(v);
+                if (j < p.n) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<float4*>(dst + c * 32 + 4 * u) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace lard

@@ -1,0 +1,161 @@
+"""ctypes binding of liblard (the C ABI declared in include/lard.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with
+their sizes and the current CUDA stream; every step of the computation runs
+in the library's kernels.  Importing this module fails loudly if the library
+has not been built.
+
+Functions keep the C names:
+    lard_kl_fwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, row_kl,
+                loss_bh=None, loss_total=None, stream=None)
+    lard_kl_bwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, grad_scale,
+                dXs, dYs, stream=None)
+    lard_device_status(stream=None) -> fault bits (raises on timeout)
+    lard_status_string(code), lard_version()
+Tensors are torch tensors [B, H, n, d] (inputs bf16 or fp32, outputs fp32),
+contiguous, on the GPU that runs the call.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblard.so")
+
+LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT = range(5)
+LARD_DTYPE_BF16, LARD_DTYPE_FP32 = 0, 1
+
+EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status", "lard_version")
+
+
+class LardError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"liblard.so is not built ({LIB_PATH}); build it with "
+            "`python -m linear_memory_attention_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, f32p, i, f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.lard_kl_fwd.restype = i
+    lib.lard_kl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, f32p, f32p, f32p, f32p, f32p, vp]
+    lib.lard_kl_bwd.restype = i
+    lib.lard_kl_bwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, f32p, f32p, f, f32p, f32p, vp]
+    lib.lard_status_string.restype = ctypes.c_char_p
+    lib.lard_status_string.argtypes = [i]
+    lib.lard_device_status.restype = i
+    lib.lard_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.lard_version.restype = i
+    lib.lard_version.argtypes = []
+    return lib
+
+
+_lib = _load()
+
+
+def _status_name(code: int) -> str:
+    return _lib.lard_status_string(int(code)).decode()
+
+
+def lard_status_string(code: int) -> str:
+    return _status_name(code)
+
+
+def lard_version() -> int:
+    return int(_lib.lard_version())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _shape(Xt):
+    import torch
+    if Xt.dim() != 4:
+        raise ValueError("inputs must be [B, H, n, d]")
+    if Xt.dtype == torch.bfloat16:
+        dt = LARD_DTYPE_BF16
+    elif Xt.dtype == torch.float32:
+        dt = LARD_DTYPE_FP32
+    else:
+        raise ValueError(f"unsupported input dtype {Xt.dtype}")
+    B, H, n, d = Xt.shape
+    return dt, int(B), int(H), int(n), int(d)
+
+
+def _check_inputs(Xt, Yt, Xs, Ys):
+    for t in (Xt, Yt, Xs, Ys):
+        if t.shape != Xt.shape or t.dtype != Xt.dtype or not t.is_contiguous():
+            raise ValueError("inputs must share one shape and dtype and be contiguous")
+
+
+def lard_kl_fwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, row_kl, loss_bh=None, loss_total=None,
+                stream=None):
+    """Phase 1: writes lse_t, lse_s, row_kl [B,H,n] and optionally loss_bh [B*H], loss_total [1]."""
+    _check_inputs(Xt, Yt, Xs, Ys)
+    dt, B, H, n, d = _shape(Xt)
+    st = _lib.lard_kl_fwd(_ptr(Xt), _ptr(Yt), _ptr(Xs), _ptr(Ys), dt, B, H, n, d, float(tau),
+                          int(bool(causal)), _ptr(lse_t), _ptr(lse_s), _ptr(row_kl), _ptr(loss_bh),
+                          _ptr(loss_total), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_fwd")
+
+
+def lard_kl_bwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, grad_scale, dXs, dYs, stream=None):
+    """Phase 2: overwrites dXs, dYs [B,H,n,d] fp32 with grad_scale * dL/dXs, dL/dYs."""
+    _check_inputs(Xt, Yt, Xs, Ys)
+    dt, B, H, n, d = _shape(Xt)
+    st = _lib.lard_kl_bwd(_ptr(Xt), _ptr(Yt), _ptr(Xs), _ptr(Ys), dt, B, H, n, d, float(tau),
+                          int(bool(causal)), _ptr(lse_t), _ptr(lse_s), float(grad_scale),
+                          _ptr(dXs), _ptr(dYs), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_bwd")
+
+
+def lard_device_status(stream=None) -> int:
+    """Synchronise the stream and check the kernels' fault word; raises on a timed-out wait."""
+    bits = ctypes.c_uint(0)
+    st = _lib.lard_device_status(_stream(stream), ctypes.byref(bits))
+    if st != LARD_OK:
+        err = LardError(st, f"lard_device_status (fault bits 0x{bits.value:x})")
+        err.fault_bits = bits.value
+        raise err
+    return bits.value
+
+
+def relation_kl(Xt, Xs, tau, causal=True, Yt=None, Ys=None, grad_scale=1.0, backward=True,
+                stream=None):
+    """Allocate the outputs and run both phases for one relation.
+
+    Returns a dict with lse_t, lse_s, row_kl, loss_bh, loss (a 1-element
+    tensor) and, if ``backward``, dXs and dYs.  Y defaults to X (self-relation).
+    """
+    import torch
+    Yt = Xt if Yt is None else Yt
+    Ys = Xs if Ys is None else Ys
+    B, H, n, d = Xt.shape
+    dev = Xt.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    out = {"lse_t": torch.empty((B, H, n), **f32), "lse_s": torch.empty((B, H, n), **f32),
+           "row_kl": torch.empty((B, H, n), **f32), "loss_bh": torch.empty((B * H,), **f32),
+           "loss": torch.empty((1,), **f32)}
+    lard_kl_fwd(Xt, Yt, Xs, Ys, tau, causal, out["lse_t"], out["lse_s"], out["row_kl"],
+                out["loss_bh"], out["loss"], stream)
+    if backward:
+        out["dXs"] = torch.empty((B, H, n, d), **f32)
+        out["dYs"] = torch.empty((B, H, n, d), **f32)
+        lard_kl_bwd(Xt, Yt, Xs, Ys, tau, causal, out["lse_t"], out["lse_s"], grad_scale,
+                    out["dXs"], out["dYs"], stream)
+    return out

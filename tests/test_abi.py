@@ -1,0 +1,93 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+include/lard.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lard.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return re.findall(r"LARD_API\s+[\w\s\*]+?\b(lard_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_memory_attention_b200 import build
+    build.build()
+    from linear_memory_attention_b200 import lard
+    return lard._lib
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for n in ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status",
+              "lard_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), f"{name} declared in include/lard.h but not exported"
+
+
+def test_binding_lists_every_export():
+    from linear_memory_attention_b200 import lard
+    assert set(declared_entry_points()) == set(lard.EXPORTS)
+
+
+def test_status_strings_and_version(lib):
+    from linear_memory_attention_b200 import lard
+    assert [lard.lard_status_string(c) for c in range(5)] == [
+        "LARD_OK", "LARD_ERR_INVALID_ARG", "LARD_ERR_UNSUPPORTED", "LARD_ERR_CUDA",
+        "LARD_ERR_TIMEOUT"]
+    assert lard.lard_status_string(99) == "LARD_ERR_UNKNOWN"
+    assert lard.lard_version() >= 100
+
+
+# Aligned fake device addresses: every case below must be rejected by the
+# argument checks, which run before any CUDA call.
+A, B_, C, D_ = 0x100000, 0x200000, 0x300000, 0x400000
+O1, O2, O3, O4, O5 = 0x10000000, 0x11000000, 0x12000000, 0x13000000, 0x14000000
+
+
+def fwd(lib, *, xt=A, yt=B_, xs=C, ys=D_, dtype=0, B=1, H=2, n=300, d=128, tau=0.088, causal=1,
+        lse_t=O1, lse_s=O2, kl=O3, loss_bh=O4, loss=O5):
+    f = ctypes.c_float
+    return lib.lard_kl_fwd(xt, yt, xs, ys, dtype, B, H, n, d, f(tau), causal, lse_t, lse_s, kl,
+                           loss_bh, loss, None)
+
+
+def bwd(lib, *, dtype=0, n=300, d=128, tau=0.088, causal=1, g=1.0, dx=O3, dy=O4, lse_t=O1,
+        lse_s=O2):
+    f = ctypes.c_float
+    return lib.lard_kl_bwd(A, B_, C, D_, dtype, 1, 2, n, d, f(tau), causal, lse_t, lse_s, f(g), dx,
+                           dy, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(xt=None), 1), (dict(ys=None), 1), (dict(lse_t=None), 1), (dict(kl=None), 1),
+    (dict(n=0), 1), (dict(B=0), 1), (dict(H=-1), 1), (dict(tau=float("nan")), 1),
+    (dict(tau=-0.5), 1), (dict(tau=0.0), 1), (dict(causal=2), 1), (dict(dtype=7), 2),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(dtype=1, d=48), 2), (dict(dtype=1, d=288), 2),
+    (dict(xs=C + 8), 1), (dict(loss_bh=None), 1), (dict(lse_s=O1), 1), (dict(kl=A), 1),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    if kw == dict(loss_bh=None):
+        # loss_total requires loss_bh
+        assert fwd(lib, loss_bh=None) == code
+    else:
+        assert fwd(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dx=None), 1), (dict(lse_s=None), 1), (dict(g=float("inf")), 1),
+    (dict(dy=O3 + 16), 1), (dict(dx=A), 1), (dict(dy=O1), 1), (dict(dx=O3 + 4), 1),
+    (dict(d=32), 2), (dict(n=-3), 1),
+])
+def test_bwd_rejects_bad_arguments(lib, kw, code):
+    assert bwd(lib, **kw) == code

@@ -1,0 +1,244 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases compare every output element by element; they span several
+128 x 128 tiles, ragged tails, n = 1 and both masks.  The five workloads are
+run at their full sizes in the launch configuration the benchmark uses; the
+oracle then checks sampled heads or sampled rows (tail rows give the exact
+dY_s of the tail columns), and properties that hold at any size are checked
+on every output.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (TOL, assert_close_abs, assert_grad_close, assert_kl_close, assert_rel,
+                         compare_full, f64, gpu_relation, grad_floor, random_cross)
+from linear_memory_attention_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lard():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from linear_memory_attention_b200 import lard as L  # fails loudly if liblard.so is missing
+    return L
+
+
+SMALL_BF16 = [(1, 1, 1, 128), (1, 2, 2, 128), (1, 2, 63, 128), (1, 2, 127, 128), (1, 2, 128, 128),
+              (1, 2, 129, 128), (2, 2, 300, 128), (1, 3, 517, 128), (1, 2, 1, 64), (1, 2, 200, 64),
+              (2, 1, 385, 64)]
+
+
+@pytest.mark.parametrize("causal", [1, 0], ids=["causal", "full"])
+@pytest.mark.parametrize("shape", SMALL_BF16, ids=lambda s: "B%dH%dn%dd%d" % s)
+def test_bf16_self_relation(lard, shape, causal):
+    B, H, n, d = shape
+    w = synth.custom(B, H, n, d, "bf16", seed=n * 7 + d, causal=bool(causal))
+    for rel in ("Q", "V"):
+        Xt, Xs = synth.make_relation(w, rel)
+        o = oracle.relation(f64(Xt), f64(Xt), f64(Xs), f64(Xs), w.tau, causal)
+        g = gpu_relation(lard, Xt, Xt, Xs, Xs, w.tau, causal)
+        compare_full(g, o, "bf16", f"{rel}/{rel} {shape} causal={causal}",
+                     grad_floor(f64(Xs), f64(Xs), w.tau, 1.0, n))
+
+
+@pytest.mark.parametrize("causal", [1, 0], ids=["causal", "full"])
+@pytest.mark.parametrize("shape", [(1, 2, 130, 128), (2, 1, 400, 64), (1, 1, 256, 128)],
+                         ids=lambda s: "B%dH%dn%dd%d" % s)
+def test_bf16_cross_relation(lard, shape, causal):
+    """X != Y for teacher and student (e.g. a Q K^T attention map)."""
+    B, H, n, d = shape
+    Xt, Yt, Xs, Ys = random_cross(B, H, n, d, "bf16", seed=n + d + causal, scale=1.3)
+    tau = 1.0 / math.sqrt(d)
+    o = oracle.relation(f64(Xt), f64(Yt), f64(Xs), f64(Ys), tau, causal)
+    g = gpu_relation(lard, Xt, Yt, Xs, Ys, tau, causal)
+    compare_full(g, o, "bf16", f"cross {shape} causal={causal}", grad_floor(f64(Xs), f64(Ys), tau, 1.0, n))
+
+
+@pytest.mark.parametrize("causal", [1, 0], ids=["causal", "full"])
+@pytest.mark.parametrize("shape", [(1, 2, 1, 64), (1, 2, 100, 64), (2, 1, 257, 128), (1, 1, 70, 32),
+                                   (1, 1, 90, 96)], ids=lambda s: "B%dH%dn%dd%d" % s)
+def test_fp32_path(lard, shape, causal):
+    B, H, n, d = shape
+    w = synth.custom(B, H, n, d, "fp32", seed=n + d, causal=bool(causal))
+    Xt, Xs = synth.make_relation(w, "K")
+    o = oracle.relation(f64(Xt), f64(Xt), f64(Xs), f64(Xs), w.tau, causal)
+    g = gpu_relation(lard, Xt, Xt, Xs, Xs, w.tau, causal)
+    compare_full(g, o, "fp32", f"fp32 {shape} causal={causal}", grad_floor(f64(Xs), f64(Xs), w.tau, 1.0, n))
+    Xt, Yt, Xs, Ys = random_cross(B, H, n, d, "fp32", seed=5 + n)
+    o = oracle.relation(f64(Xt), f64(Yt), f64(Xs), f64(Ys), w.tau, causal)
+    g = gpu_relation(lard, Xt, Yt, Xs, Ys, w.tau, causal)
+    compare_full(g, o, "fp32", f"fp32 cross {shape} causal={causal}", grad_floor(f64(Xs), f64(Ys), w.tau, 1.0, n))
+
+
+def test_grad_scale_and_identical_student(lard):
+    w = synth.custom(1, 2, 300, 128, "bf16", seed=9)
+    Xt, Xs = synth.make_relation(w, "Q")
+    o = oracle.relation(f64(Xt), f64(Xt), f64(Xs), f64(Xs), w.tau, True)
+    g = gpu_relation(lard, Xt, Xt, Xs, Xs, w.tau, True, grad_scale=-0.37)
+    assert_grad_close(g["dXs"], -0.37 * o["dXs"], 1e-2, "scaled dXs")
+    assert_grad_close(g["dYs"], -0.37 * o["dYs"], 1e-2, "scaled dYs")
+    # student == teacher: KL and gradients vanish (up to the rounding of exp)
+    g = gpu_relation(lard, Xt, Xt, Xt.clone(), Xt.clone(), w.tau, True)
+    assert np.abs(g["row_kl"]).max() <= 1e-5
+    scale = np.abs(o["dXs"]).max()
+    assert np.abs(g["dXs"]).max() <= 1e-4 * scale and np.abs(g["dYs"]).max() <= 1e-4 * scale
+
+
+def test_causal_row0_and_determinism(lard):
+    w = synth.custom(2, 2, 700, 128, "bf16", seed=4)
+    Xt, Xs = synth.make_relation(w, "K")
+    g1 = gpu_relation(lard, Xt, Xt, Xs, Xs, w.tau, True)
+    g2 = gpu_relation(lard, Xt, Xt, Xs, Xs, w.tau, True)
+    assert np.abs(g1["row_kl"][..., 0]).max() <= 1e-6, "row 0 has a single entry: KL must be 0"
+    z00 = w.tau * (f64(Xs)[..., 0, :] ** 2).sum(-1)
+    assert_close_abs(g1["lse_s"][..., 0], z00, 1e-3, "LSE(0) = Z(0,0)")
+    for k in ("lse_t", "lse_s", "row_kl", "loss", "dYs"):
+        assert np.array_equal(g1[k], g2[k]), f"{k} must be bitwise reproducible"
+
+
+def test_extra_memory_is_linear(lard):
+    """The library allocates nothing: device free memory is unchanged by a call."""
+    w = synth.custom(1, 8, 4096, 128, "bf16", seed=1)
+    Xt, Xs = (t.cuda() for t in synth.make_relation(w, "Q"))
+    lard.relation_kl(Xt, Xs, w.tau)
+    torch.cuda.synchronize()
+    B, H, n, d = Xt.shape
+    f32 = dict(device="cuda", dtype=torch.float32)
+    bufs = [torch.empty((B, H, n), **f32) for _ in range(3)] + [torch.empty((B * H,), **f32),
+                                                                torch.empty((1,), **f32)]
+    gx, gy = torch.empty((B, H, n, d), **f32), torch.empty((B, H, n, d), **f32)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    lard.lard_kl_fwd(Xt, Xt, Xs, Xs, w.tau, True, *bufs)
+    lard.lard_kl_bwd(Xt, Xt, Xs, Xs, w.tau, True, bufs[0], bufs[1], 1.0, gx, gy)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert abs(free0 - free1) < (2 << 20), "a call must not allocate device memory"
+
+
+# ------------------------------------------------------------------ workloads at full size
+
+def _run_workload(lard, w, check):
+    """Run every relation of a workload through the C ABI (one at a time, so
+    that host and device memory stay bounded) and hand each to ``check``."""
+    for rel in w.relations:
+        Xt, Xs = synth.make_relation(w, rel)
+        xt, xs = Xt.cuda(), Xs.cuda()
+        g = lard.relation_kl(xt, xs, w.tau, w.causal)
+        torch.cuda.synchronize()
+        lard.lard_device_status()
+        _properties(xs, g, w, f"{w.name} {rel}")
+        check(rel, Xt, Xs, g)
+        del g, xt, xs
+        torch.cuda.empty_cache()
+
+
+def _properties(xs, g, w, what):
+    """Checks that hold at any size, on every output (computed on the device in fp64)."""
+    dX, dY = g["dXs"].double(), g["dYs"].double()
+    assert torch.isfinite(dX).all() and torch.isfinite(dY).all(), what + ": non-finite gradients"
+    kl = g["row_kl"].double()
+    assert kl.min().item() >= -1e-4, f"{what}: KL must be non-negative"
+    torch.testing.assert_close(g["loss_bh"].double(), kl.reshape(-1, w.n).mean(-1), rtol=1e-5, atol=1e-9)
+    assert_rel(g["loss"].item(), g["loss_bh"].double().sum().item(), 1e-5, what + " loss total")
+    x = xs.double()
+    zdiag = w.tau * (x * x).sum(-1)
+    assert bool((g["lse_s"].double() >= zdiag - 1e-3).all()), f"{what}: LSE_s below the diagonal logit"
+    # sum_i <dX_s[i], X_s[i]> = sum_j <dY_s[j], Y_s[j]> (both equal sum_ij dZ Z_s), per head
+    lhs = (dX * x).sum(dim=(-1, -2))
+    rhs = (dY * x).sum(dim=(-1, -2))
+    scale = (dX * x).abs().sum(dim=(-1, -2))
+    assert bool(((lhs - rhs).abs() <= 2e-2 * scale + 1e-9).all()), f"{what}: duality violated"
+
+
+def _host(t):
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def _check_heads(w, heads):
+    tol = TOL[w.dtype]
+
+    def check(rel, Xt, Xs, g):
+        H = Xt.shape[1]
+        for (b, h) in heads[rel]:
+            xt, xs = f64(Xt[b, h]), f64(Xs[b, h])
+            o = oracle.relation(xt, xt, xs, xs, w.tau, w.causal)
+            what = f"{w.name} {rel} head ({b},{h})"
+            assert_close_abs(_host(g["lse_t"][b, h]), o["lse_t"], tol["lse"], what + " lse_t")
+            assert_close_abs(_host(g["lse_s"][b, h]), o["lse_s"], tol["lse"], what + " lse_s")
+            assert_kl_close(_host(g["row_kl"][b, h]), o["row_kl"], tol, what + " row_kl")
+            assert_rel(g["loss_bh"][b * H + h].item(), o["loss"], tol["loss"], what + " loss", tol["loss_abs"])
+            floor = grad_floor(xs, xs, w.tau, 1.0, w.n)
+            assert_grad_close(_host(g["dXs"][b, h]), o["dXs"], tol["grad"], what + " dXs", floor)
+            assert_grad_close(_host(g["dYs"][b, h]), o["dYs"], tol["grad"], what + " dYs", floor)
+    return check
+
+
+def _check_rows(w, heads, n_tail, n_random, seed):
+    """Tail rows [n - n_tail, n) (with the exact dY_s of the tail columns) and
+    random earlier rows, against the oracle's rows mode.  The gradient bound
+    uses the largest oracle gradient over all sampled rows of the head."""
+    tol = TOL[w.dtype]
+    rng = np.random.default_rng(seed)
+    n = w.n
+
+    def check(rel, Xt, Xs, g):
+        for (b, h) in heads[rel]:
+            xt, xs = f64(Xt[b, h]), f64(Xs[b, h])
+            what = f"{w.name} {rel} head ({b},{h})"
+            floor = grad_floor(xs, xs, w.tau, 1.0, n)
+            r0 = n - n_tail
+            o = oracle.rows(xt, xt, xs, xs, w.tau, w.causal, r0, n, want_dY=True)
+            assert_grad_close(_host(g["dYs"][b, h, r0:]), o["dYs"][r0:], tol["grad"], what + " tail-column dYs", floor)
+            rows = np.concatenate([np.sort(rng.choice(r0, size=min(n_random, r0), replace=False)),
+                                   np.arange(r0, n)]).astype(int)
+            o_lt, o_ls, o_kl, o_dx = [], [], [], []
+            for i in rows[:-n_tail]:
+                oi = oracle.rows(xt, xt, xs, xs, w.tau, w.causal, int(i), int(i) + 1)
+                o_lt.append(oi["lse_t"]), o_ls.append(oi["lse_s"]), o_kl.append(oi["row_kl"]), o_dx.append(oi["dXs"])
+            o_lt.append(o["lse_t"]), o_ls.append(o["lse_s"]), o_kl.append(o["row_kl"]), o_dx.append(o["dXs"])
+            idx = torch.as_tensor(rows)
+            assert_close_abs(_host(g["lse_t"][b, h][idx]), np.concatenate(o_lt), tol["lse"], what + " sampled lse_t")
+            assert_close_abs(_host(g["lse_s"][b, h][idx]), np.concatenate(o_ls), tol["lse"], what + " sampled lse_s")
+            assert_kl_close(_host(g["row_kl"][b, h][idx]), np.concatenate(o_kl), tol, what + " sampled row_kl")
+            assert_grad_close(_host(g["dXs"][b, h][idx]), np.concatenate(o_dx), tol["grad"], what + " sampled dXs", floor)
+    return check
+
+
+def test_workload_fp32_small(lard):
+    w = synth.WORKLOADS["fp32-small"]
+
+    def check(rel, Xt, Xs, g):
+        o = oracle.relation(f64(Xt), f64(Xt), f64(Xs), f64(Xs), w.tau, True)
+        compare_full({k: _host(v) for k, v in g.items()}, o, "fp32", f"{w.name} {rel}",
+                     grad_floor(f64(Xs), f64(Xs), w.tau, 1.0, w.n))
+    _run_workload(lard, w, check)
+
+
+def test_workload_n4096(lard):
+    w = synth.WORKLOADS["n4096"]
+    _run_workload(lard, w, _check_heads(w, {r: [(0, 0), (0, 31)] for r in w.relations}))
+
+
+def test_workload_gqa_n8000(lard):
+    w = synth.WORKLOADS["gqa-n8000"]
+    heads = {"Q": [(0, 3), (1, 30)], "K": [(0, 0), (1, 7)], "V": [(1, 2)]}
+    _run_workload(lard, w, _check_rows(w, heads, n_tail=200, n_random=24, seed=5))
+
+
+def test_workload_n16384(lard):
+    w = synth.WORKLOADS["n16384"]
+    _run_workload(lard, w, _check_rows(w, {r: [(0, 5)] for r in w.relations}, n_tail=160,
+                                       n_random=16, seed=6))
+
+
+def test_workload_n32768(lard):
+    w = synth.WORKLOADS["n32768"]
+    _run_workload(lard, w, _check_rows(w, {r: [(0, 0), (0, 17)] for r in w.relations}, n_tail=160,
+                                       n_random=16, seed=7))
