@@ -121,6 +121,19 @@ bool make_map(CUtensorMap* m, const void* base, long long BH, int n, int d) {
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tensor map over the fp32 gradient [BH, n, d] with 32 x 32 boxes
+// (128-byte rows), 128-byte swizzle, for the TMA reduce-adds of Phase 2.
+bool make_grad_map(CUtensorMap* m, void* base, long long BH, int n, int d) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(n) * d * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Checks shared by both phases.
 lard_status check_common(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
                          int B, int H, int n, int d, float tau, int causal, long long* BH_out) {
@@ -269,9 +282,9 @@ lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const vo
     const int T = (n + 127) / 128;
     const double dz_scale = static_cast<double>(tau) * grad_scale / n;
     if (dtype == LARD_DTYPE_BF16) {
-        CUtensorMap mxt, myt, mxs, mys;
+        CUtensorMap mxt, myt, mxs, mys, mdx;
         if (!make_map(&mxt, Xt, BH, n, d) || !make_map(&myt, Yt, BH, n, d) || !make_map(&mxs, Xs, BH, n, d) ||
-            !make_map(&mys, Ys, BH, n, d))
+            !make_map(&mys, Ys, BH, n, d) || !make_grad_map(&mdx, dXs, BH, n, d))
             return LARD_ERR_INVALID_ARG;
         if (cudaMemsetAsync(dXs, 0, ngrad, stream) != cudaSuccess) return LARD_ERR_CUDA;
         lard::TcBwdParams p;
@@ -283,14 +296,13 @@ lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const vo
         p.dz_scale = static_cast<float>(dz_scale);
         p.lse_t = lse_t;
         p.lse_s = lse_s;
-        p.dXs = dXs;
         p.dYs = dYs;
         p.wait_ns = kWaitLimitNs;
         const unsigned grid = static_cast<unsigned>(BH * T);
         if (d == 128)
-            lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+            lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, mdx, p);
         else
-            lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+            lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, mdx, p);
     } else {
         lard::Fp32Params p;
         p.BH = static_cast<int>(BH);

@@ -8,17 +8,21 @@
 //
 // One CTA owns a 128-column block J of one (batch, head); its dY_s[J]
 // accumulator stays in TMEM for the whole sweep over the row blocks I >= J
-// (all I without the mask), and each tile's dX_s[I] contribution is added
-// to HBM with fp32 vector atomics.
+// (all I without the mask).  Each tile's dX_s[I] contribution is staged in
+// shared memory and added to HBM with TMA bulk reduce-adds (fp32 adds in L2,
+// whole 128-byte lines, rows past n clipped by the tensor map).
 // TMEM (512 columns): dY [0, D), S_t [128, 256), S_s [256, 384), dX [384, 384 + D).
-// Shared memory: Y_t[J], Y_s[J] resident; a 2-stage ring of (X_t[I], X_s[I]);
-// one 128 x 128 bf16 dZ tile, 128B-swizzled, read by both gradient GEMMs:
+// Shared memory: Y_t[J], Y_s[J] resident; a 2-stage ring for X_s[I]; one
+// buffer for X_t[I] (only the first GEMM of a tile reads it, so the next one
+// has a whole tile of softmax work to land); one 128 x 128 bf16 dZ tile,
+// 128B-swizzled, read by both gradient GEMMs:
 //   GEMM 3  dY[J] += dZ^T X_s[I]   (A = dZ as MN-major, B = X_s as MN-major)
 //   GEMM 4  dX[I]  = dZ  Y_s[J]    (A = dZ as K-major,  B = Y_s as MN-major)
+// and 2 x 4 KB of dX staging per drain warp.
 // Roles (512 threads):
 //   warp 0       TMA producer          warp 1   TMEM owner, MMA issuer
 //   warps 4-11   dZ: one row per thread, one 64-column half per warpgroup
-//   warps 12-15  dX drain (TMEM -> red.global.add) and the final dY store
+//   warps 12-15  dX drain (TMEM -> smem -> TMA reduce-add), final dY store
 #pragma once
 
 #include "lard_kernel_common.cuh"
@@ -31,7 +35,6 @@ struct TcBwdParams {
     float dz_scale;  // tau * grad_scale / n: dZ and the chain-rule tau in one factor
     const float* lse_t;
     const float* lse_s;
-    float* dXs;
     float* dYs;
     unsigned long long wait_ns;
 };
@@ -40,20 +43,22 @@ template <int D>
 struct BwdLayout {
     static constexpr int KC = D / 64;
     static constexpr int TILE = KC * 16384;
-    static constexpr int NS = 2;
     static constexpr int OFF_YT = 0;
     static constexpr int OFF_YS = TILE;
-    static constexpr int OFF_X = 2 * TILE;  // stage s: X_t at OFF_X + 2*s*TILE, X_s after it
-    static constexpr int OFF_DZ = OFF_X + NS * 2 * TILE;
-    static constexpr int OFF_CTRL = OFF_DZ + 32768;
+    static constexpr int OFF_XS = 2 * TILE;  // 2 stages
+    static constexpr int OFF_XT = 4 * TILE;  // 1 stage
+    static constexpr int OFF_DZ = 5 * TILE;
+    static constexpr int OFF_STG = OFF_DZ + 32768;  // 4 drain warps x 2 x 4 KB
+    static constexpr int OFF_CTRL = OFF_STG + 32768;
     static constexpr int CTRL_BYTES = 1024;
     static constexpr int SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;
 };
 
 struct BwdCtrl {
     uint64_t y_full;
-    uint64_t x_full[2];
-    uint64_t x_empty[2];
+    uint64_t xs_full[2];
+    uint64_t xs_empty[2];
+    uint64_t xt_full, xt_empty;
     uint64_t s_full, s_free, dz_full, dz_free, dx_full, dx_free, dy_full, mma_done;
     uint32_t tmem_base;
     int abort_flag;
@@ -67,7 +72,8 @@ __global__ void __launch_bounds__(512, 1)
     lard_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_xt,
                        const __grid_constant__ CUtensorMap tm_yt,
                        const __grid_constant__ CUtensorMap tm_xs,
-                       const __grid_constant__ CUtensorMap tm_ys, const TcBwdParams p) {
+                       const __grid_constant__ CUtensorMap tm_ys,
+                       const __grid_constant__ CUtensorMap tm_dx, const TcBwdParams p) {
     using L = BwdLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -85,10 +91,12 @@ __global__ void __launch_bounds__(512, 1)
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(&ctrl->y_full, 1);
-        for (int s = 0; s < L::NS; ++s) {
-            ptx::mbar_init(&ctrl->x_full[s], 1);
-            ptx::mbar_init(&ctrl->x_empty[s], 1);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(&ctrl->xs_full[s], 1);
+            ptx::mbar_init(&ctrl->xs_empty[s], 1);
         }
+        ptx::mbar_init(&ctrl->xt_full, 1);
+        ptx::mbar_init(&ctrl->xt_empty, 1);
         ptx::mbar_init(&ctrl->s_full, 1);
         ptx::mbar_init(&ctrl->s_free, 8);
         ptx::mbar_init(&ctrl->dz_full, 8);
@@ -105,6 +113,7 @@ __global__ void __launch_bounds__(512, 1)
         ptx::prefetch_tensormap(&tm_yt);
         ptx::prefetch_tensormap(&tm_xs);
         ptx::prefetch_tensormap(&tm_ys);
+        ptx::prefetch_tensormap(&tm_dx);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&ctrl->tmem_base, 512);
@@ -126,28 +135,40 @@ __global__ void __launch_bounds__(512, 1)
             }
         }
         __syncwarp();
-        int issued = 0;
+        int issued_t = 0, issued_s = 0;
         for (int k = 0; k < K; ++k) {
-            const int s = k & 1, rnd = k >> 1;
-            bool ok = ptx::mbar_wait(&ctrl->x_empty[s], (rnd & 1) ^ 1, abort_flag, lim, &g_lard_fault,
+            const int I = row_block(k);
+            // X_t(k) may land once S_t(k-1) has been computed ...
+            bool ok = ptx::mbar_wait(&ctrl->xt_empty, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault,
                                      kFaultBwdProducer);
             if (!__all_sync(0xffffffffu, ok)) break;
             if (lane == 0) {
-                const int I = row_block(k);
-                uint8_t* xt = smem + L::OFF_X + 2 * s * L::TILE;
-                ptx::mbar_arrive_expect_tx(&ctrl->x_full[s], 2 * L::TILE);
-                for (int c = 0; c < L::KC; ++c) {
-                    ptx::tma_load_3d(xt + c * 16384, &tm_xt, &ctrl->x_full[s], c * 64, I * 128, bh);
-                    ptx::tma_load_3d(xt + L::TILE + c * 16384, &tm_xs, &ctrl->x_full[s], c * 64, I * 128, bh);
-                }
+                ptx::mbar_arrive_expect_tx(&ctrl->xt_full, L::TILE);
+                for (int c = 0; c < L::KC; ++c)
+                    ptx::tma_load_3d(smem + L::OFF_XT + c * 16384, &tm_xt, &ctrl->xt_full, c * 64, I * 128, bh);
             }
             __syncwarp();
-            ++issued;
+            ++issued_t;
+            // ... and X_s(k) once GEMM 3 of tile k-2 has released its stage.
+            const int s = k & 1;
+            ok = ptx::mbar_wait(&ctrl->xs_empty[s], ((k >> 1) & 1) ^ 1, abort_flag, lim, &g_lard_fault,
+                                kFaultBwdProducer);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (lane == 0) {
+                ptx::mbar_arrive_expect_tx(&ctrl->xs_full[s], L::TILE);
+                for (int c = 0; c < L::KC; ++c)
+                    ptx::tma_load_3d(smem + L::OFF_XS + s * L::TILE + c * 16384, &tm_xs, &ctrl->xs_full[s],
+                                     c * 64, I * 128, bh);
+            }
+            __syncwarp();
+            ++issued_s;
         }
+        // Let every copy this warp started land before the block can exit.
         ptx::mbar_drain(&ctrl->y_full, 0, lim);
-        for (int s = 0; s < L::NS && s < issued; ++s) {
-            const int last = s + L::NS * ((issued - 1 - s) / L::NS);
-            ptx::mbar_drain(&ctrl->x_full[s], (last / L::NS) & 1, lim);
+        if (issued_t > 0) ptx::mbar_drain(&ctrl->xt_full, (issued_t - 1) & 1, lim);
+        for (int s = 0; s < 2 && s < issued_s; ++s) {
+            const int last = s + 2 * ((issued_s - 1 - s) / 2);
+            ptx::mbar_drain(&ctrl->xs_full[s], (last >> 1) & 1, lim);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -156,40 +177,55 @@ __global__ void __launch_bounds__(512, 1)
         constexpr uint32_t kIdescDX = ptx::idesc_bf16(128, D, 0, 1);
         const uint32_t syt = ptx::smem_u32(smem + L::OFF_YT);
         const uint32_t sys = ptx::smem_u32(smem + L::OFF_YS);
+        const uint32_t sxt = ptx::smem_u32(smem + L::OFF_XT);
         const uint32_t sdz = ptx::smem_u32(smem + L::OFF_DZ);
-        auto issue_s = [&](int k) {
-            const uint32_t sxt = ptx::smem_u32(smem + L::OFF_X + 2 * (k & 1) * L::TILE);
-            const uint32_t sxs = sxt + L::TILE;
+        auto sxs = [&](int k) { return ptx::smem_u32(smem + L::OFF_XS + (k & 1) * L::TILE); };
+        auto issue_ss = [&](int k) {
+            const uint32_t a = sxs(k);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+                ptx::umma_bf16(tmem + kTmemSs, ptx::sdesc_sw128(a + koff, 16, 1024),
+                               ptx::sdesc_sw128(sys + koff, 16, 1024), kIdescS, kk > 0);
+            }
+        };
+        auto issue_st = [&]() {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
                 ptx::umma_bf16(tmem + kTmemSt, ptx::sdesc_sw128(sxt + koff, 16, 1024),
                                ptx::sdesc_sw128(syt + koff, 16, 1024), kIdescS, kk > 0);
             }
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                ptx::umma_bf16(tmem + kTmemSs, ptx::sdesc_sw128(sxs + koff, 16, 1024),
-                               ptx::sdesc_sw128(sys + koff, 16, 1024), kIdescS, kk > 0);
-            }
+            ptx::umma_commit(&ctrl->xt_empty);
             ptx::umma_commit(&ctrl->s_full);
         };
+        // S(k) for k = 0: S_s first (X_s(0) is loaded before X_t(0) is needed).
         bool ok = ptx::mbar_wait(&ctrl->y_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma) &&
-                  ptx::mbar_wait(&ctrl->x_full[0], 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
+                  ptx::mbar_wait(&ctrl->xs_full[0], 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma) &&
+                  ptx::mbar_wait(&ctrl->xt_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             ptx::tc_fence_after();
-            if (lane == 0) issue_s(0);
+            if (lane == 0) {
+                issue_ss(0);
+                issue_st();
+            }
             __syncwarp();
         }
         for (int k = 0; ok && k < K; ++k) {
             if (k + 1 < K) {
-                ok = ptx::mbar_wait(&ctrl->x_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag, lim,
+                // S(k+1) as soon as the dZ warps have read S(k) out of TMEM.
+                ok = ptx::mbar_wait(&ctrl->xs_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag, lim,
                                     &g_lard_fault, kFaultBwdMma) &&
                      ptx::mbar_wait(&ctrl->s_free, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 ptx::tc_fence_after();
-                if (lane == 0) issue_s(k + 1);
+                if (lane == 0) issue_ss(k + 1);
+                __syncwarp();
+                ok = ptx::mbar_wait(&ctrl->xt_full, (k + 1) & 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                ptx::tc_fence_after();
+                if (lane == 0) issue_st();
                 __syncwarp();
             }
             ok = ptx::mbar_wait(&ctrl->dz_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdMma) &&
@@ -197,12 +233,12 @@ __global__ void __launch_bounds__(512, 1)
             if (!__all_sync(0xffffffffu, ok)) break;
             ptx::tc_fence_after();
             if (lane == 0) {
-                const uint32_t sxs = ptx::smem_u32(smem + L::OFF_X + 2 * (k & 1) * L::TILE) + L::TILE;
+                const uint32_t b3 = sxs(k);
                 // GEMM 3: dY[J] (+)= dZ^T X_s[I]; K runs over the 128 rows i, 16 per step.
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     ptx::umma_bf16(tmem + kTmemDY, ptx::sdesc_sw128(sdz + kk * 2048, 16384, 1024),
-                                   ptx::sdesc_sw128(sxs + kk * 2048, 16384, 1024), kIdescDY,
+                                   ptx::sdesc_sw128(b3 + kk * 2048, 16384, 1024), kIdescDY,
                                    (k > 0 || kk > 0) ? 1u : 0u);
                 // GEMM 4: dX[I] = dZ Y_s[J]; K runs over the 128 columns j.
 #pragma unroll
@@ -212,7 +248,7 @@ __global__ void __launch_bounds__(512, 1)
                                    ptx::sdesc_sw128(sys + kk * 2048, 16384, 1024), kIdescDX,
                                    kk > 0 ? 1u : 0u);
                 ptx::umma_commit(&ctrl->dz_free);
-                ptx::umma_commit(&ctrl->x_empty[k & 1]);
+                ptx::umma_commit(&ctrl->xs_empty[k & 1]);
                 ptx::umma_commit(&ctrl->dx_full);
             }
             __syncwarp();
@@ -249,7 +285,7 @@ __global__ void __launch_bounds__(512, 1)
             const float bt = row_ok ? nlt * kLog2e : 0.f;
             const float bs = row_ok ? nls * kLog2e : 0.f;
             if (k + 1 < K) load_lse(k + 1, nlt, nls);
-            int jlim = 128;
+            int jlim = 128;  // columns [0, jlim) of this tile are allowed for row i
             if (!row_ok) jlim = 0;
             else if (p.causal) { if (I == J) jlim = r + 1; }
             else if (J == p.T - 1) jlim = p.n - J * 128;
@@ -298,29 +334,48 @@ __global__ void __launch_bounds__(512, 1)
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        uint8_t* stage = smem + L::OFF_STG + q * 8192;  // this warp's two 4 KB boxes
+        const uint32_t stage_u32 = ptx::smem_u32(stage);
+        int nchunk = 0;
         bool ok = true;
         for (int k = 0; k < K; ++k) {
-            const int i = row_block(k) * 128 + r;
+            const int y0 = row_block(k) * 128 + q * 32;  // first dX row of this warp's box
             ok = ptx::mbar_wait(&ctrl->dx_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdEpilogue);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            float* dst = p.dXs + (static_cast<size_t>(bh) * p.n + (i < p.n ? i : 0)) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float v[32];
                 __syncwarp();
                 ptx::tmem_ld32(lane_base + kTmemDX + c * 32, v);
                 ptx::tmem_ld_wait(v);
-                if (i < p.n) {
+                if (c == D / 32 - 1) {  // the dX accumulator is free for the next tile
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&ctrl->dx_free);
+                }
+                if (y0 < p.n) {  // warp-uniform: a box wholly past n is skipped
+                    const int b = nchunk & 1;
+                    ++nchunk;
+                    if (lane == 0) ptx::bulk_wait_read<1>();  // box b's previous reduce has read it
+                    __syncwarp();
+                    const uint32_t row = stage_u32 + b * 4096 + lane * 128;
+                    const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
-                        ptx::red_add_v4(dst + c * 32 + 4 * u, v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        ptx::st_shared_v4(row + ((u ^ (lane & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
+                                          w[4 * u + 3]);
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_reduce_add_3d(&tm_dx, stage + b * 4096, c * 32, y0, bh);
+                        ptx::bulk_commit();
+                    }
                 }
             }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&ctrl->dx_free);
         }
+        if (lane == 0) ptx::bulk_wait<0>();
+        __syncwarp();
         if (ok) {
             ok = ptx::mbar_wait(&ctrl->dy_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdEpilogue);
             ok = __all_sync(0xffffffffu, ok);
