@@ -63,6 +63,17 @@ cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// The warp-specialised kernels move registers between warpgroups with
+// setmaxnreg; that only terminates if the block's launch allocation covers
+// every warpgroup's share.  Checks the built kernel's register count.
+template <typename K>
+bool split_fits(K kernel, int threads, int split_total) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return false;
+    const int per_thread = (a.numRegs + 7) / 8 * 8;
+    return per_thread * threads >= split_total;
+}
+
 // One-time setup of device `dev` (made current by the caller).
 lard_status setup_device(int dev) {
     std::lock_guard<std::mutex> lk(g_mu);
@@ -90,6 +101,13 @@ lard_status setup_device(int dev) {
                   set_smem(lard::lard_bwd_tc_kernel<64>, lard::BwdLayout<64>::SMEM_BYTES) == cudaSuccess &&
                   set_smem(lard::lard_bwd_tc_kernel<128>, lard::BwdLayout<128>::SMEM_BYTES) == cudaSuccess;
         if (!ok) st = LARD_ERR_CUDA;
+    }
+    if (st == LARD_OK) {
+        const bool fits = split_fits(lard::lard_fwd_tc_kernel<64>, 384, lard::kFwdRegsSplitTotal) &&
+                          split_fits(lard::lard_fwd_tc_kernel<128>, 384, lard::kFwdRegsSplitTotal) &&
+                          split_fits(lard::lard_bwd_tc_kernel<64>, 512, lard::kBwdRegsSplitTotal) &&
+                          split_fits(lard::lard_bwd_tc_kernel<128>, 512, lard::kBwdRegsSplitTotal);
+        if (!fits) st = LARD_ERR_UNSUPPORTED;  // a build whose register count cannot host the split
     }
     g_dev_status[dev] = st;
     g_ready[dev] = true;

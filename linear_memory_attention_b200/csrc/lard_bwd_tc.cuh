@@ -67,6 +67,15 @@ static_assert(sizeof(BwdCtrl) <= 1024, "control block too large");
 
 constexpr uint32_t kTmemDY = 0, kTmemSt = 128, kTmemSs = 256, kTmemDX = 384;
 
+// Register split (per thread): launched at 128; the control warpgroup and the
+// drain warpgroup give registers to the two dZ warpgroups.  The shares must
+// not add up to more than the launch allocation, or setmaxnreg.inc would wait
+// for ever; the host checks the built kernel's register count against
+// kBwdRegsSplitTotal before the first launch.
+constexpr int kBwdRegsLaunch = 128, kBwdRegsCtl = 72, kBwdRegsDz = 184, kBwdRegsDrain = 64;
+constexpr int kBwdRegsSplitTotal = 128 * (kBwdRegsCtl + kBwdRegsDrain + 2 * kBwdRegsDz);
+static_assert(kBwdRegsSplitTotal <= 512 * kBwdRegsLaunch, "register split exceeds the launch allocation");
+
 template <int D>
 __global__ void __launch_bounds__(512, 1)
     lard_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_xt,
@@ -124,8 +133,9 @@ __global__ void __launch_bounds__(512, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
     const uint64_t lim = p.wait_ns;
-
-    if (warp == 0) {
+    if (warp < 4) {
+      ptx::regs_dec<kBwdRegsCtl>();
+      if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&ctrl->y_full, 2 * L::TILE);
@@ -170,7 +180,7 @@ __global__ void __launch_bounds__(512, 1)
             const int last = s + 2 * ((issued_s - 1 - s) / 2);
             ptx::mbar_drain(&ctrl->xs_full[s], (last >> 1) & 1, lim);
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t kIdescS = ptx::idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t kIdescDY = ptx::idesc_bf16(128, D, 1, 1);
@@ -259,7 +269,9 @@ __global__ void __launch_bounds__(512, 1)
         }
         __syncwarp();
         ptx::mbar_drain(&ctrl->mma_done, 0, lim);
-    } else if (warp >= 4 && warp < 12) {
+      }
+    } else if (warp < 12) {
+        ptx::regs_inc<kBwdRegsDz>();
         // ------------------------------------------------------------ dZ
         const int q = warp & 3;
         const int hcol = (warp - 4) >> 2;
@@ -293,21 +305,27 @@ __global__ void __launch_bounds__(512, 1)
             bool ok = ptx::mbar_wait(&ctrl->s_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdSoftmax);
             if (!__all_sync(0xffffffffu, ok)) break;
             ptx::tc_fence_after();
-            uint32_t pk[32];
+            // Read this thread's 64 columns of S_t and S_s at once and hand the
+            // TMEM back, so that S(k+1) can be computed under this tile's math.
+            float st0[32], ss0[32], st1[32], ss1[32];
+            __syncwarp();
+            ptx::tmem_ld32(lane_base + kTmemSt + hcol * 64, st0);
+            ptx::tmem_ld32(lane_base + kTmemSs + hcol * 64, ss0);
+            ptx::tmem_ld32(lane_base + kTmemSt + hcol * 64 + 32, st1);
+            ptx::tmem_ld32(lane_base + kTmemSs + hcol * 64 + 32, ss1);
+            ptx::tmem_ld_wait(st0);
+            ptx::reg_dep(ss0);
+            ptx::reg_dep(st1);
+            ptx::reg_dep(ss1);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ctrl->s_free);
 #pragma unroll
             for (int round = 0; round < 2; ++round) {
                 const int cb = hcol * 64 + round * 32;
-                float st[32], ss[32];
-                __syncwarp();
-                ptx::tmem_ld32(lane_base + kTmemSt + cb, st);
-                ptx::tmem_ld32(lane_base + kTmemSs + cb, ss);
-                ptx::tmem_ld_wait(st);
-                ptx::reg_dep(ss);
-                if (round == 1) {
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&ctrl->s_free);
-                }
+                const float* st = round ? st1 : st0;
+                const float* ss = round ? ss1 : ss0;
+                uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float rt0 = ptx::ex2(fmaf(st[c], cf, -bt));
@@ -316,20 +334,27 @@ __global__ void __launch_bounds__(512, 1)
                     const float rs1 = ptx::ex2(fmaf(ss[c + 1], cf, -bs));
                     const float d0 = (cb + c < jlim) ? (rs0 - rt0) * dzs : 0.f;
                     const float d1 = (cb + c + 1 < jlim) ? (rs1 - rt1) * dzs : 0.f;
-                    pk[round * 16 + (c >> 1)] = ptx::pack_bf16x2(d0, d1);
+                    pk[c >> 1] = ptx::pack_bf16x2(d0, d1);
+                }
+                if (round == 0) {  // the dZ tile of k-1 must have been consumed by GEMMs 3 and 4
+                    ok = ptx::mbar_wait(&ctrl->dz_free, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault,
+                                        kFaultBwdSoftmax);
+                    if (!__all_sync(0xffffffffu, ok)) break;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int unit = round * 4 + u;
+                    ptx::st_shared_v4(sdz_row + ((unit ^ (r & 7)) << 4), pk[4 * u], pk[4 * u + 1],
+                                      pk[4 * u + 2], pk[4 * u + 3]);
                 }
             }
-            ok = ptx::mbar_wait(&ctrl->dz_free, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault, kFaultBwdSoftmax);
-            if (!__all_sync(0xffffffffu, ok)) break;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                ptx::st_shared_v4(sdz_row + ((u ^ (r & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                                  pk[4 * u + 3]);
+            if (!ok) break;
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&ctrl->dz_full);
         }
-    } else if (warp >= 12) {
+    } else {
+        ptx::regs_dec<kBwdRegsDrain>();
         // ------------------------------------------------------------ dX drain, dY store
         const int q = warp & 3;
         const int r = q * 32 + lane;

@@ -49,6 +49,15 @@ struct FwdLayout {
     static constexpr int SMEM_BYTES = OFF_CTRL + CTRL_BYTES + 1024;  // + alignment slack
 };
 
+// Register split (per thread): launched at 168; the control warpgroup gives
+// registers to the two statistics warpgroups.  The shares must not add up to
+// more than the launch allocation, or setmaxnreg.inc would wait for ever; the
+// host checks the built kernel's register count against kFwdRegsSplitTotal
+// before the first launch.
+constexpr int kFwdRegsLaunch = 168, kFwdRegsCtl = 40, kFwdRegsStat = 232;
+constexpr int kFwdRegsSplitTotal = 128 * (kFwdRegsCtl + 2 * kFwdRegsStat);
+static_assert(kFwdRegsSplitTotal <= 384 * kFwdRegsLaunch, "register split exceeds the launch allocation");
+
 struct FwdCtrl {
     uint64_t x_full;
     uint64_t y_full[4];
@@ -112,8 +121,9 @@ __global__ void __launch_bounds__(384, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
     const uint64_t lim = p.wait_ns;
-
-    if (warp == 0) {
+    if (warp < 4) {
+      ptx::regs_dec<kFwdRegsCtl>();
+      if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&ctrl->x_full, 2 * L::TILE);
@@ -147,7 +157,7 @@ __global__ void __launch_bounds__(384, 1)
             const int last = s + L::NS * ((issued - 1 - s) / L::NS);
             ptx::mbar_drain(&ctrl->y_full[s], (last / L::NS) & 1, lim);
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 128, 0, 0);
         const uint32_t sxt = ptx::smem_u32(smem + L::OFF_XT);
@@ -188,7 +198,9 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) ptx::umma_commit(&ctrl->mma_done);
         __syncwarp();
         ptx::mbar_drain(&ctrl->mma_done, 0, lim);
-    } else if (warp >= 4) {
+      }
+    } else {
+        ptx::regs_inc<kFwdRegsStat>();
         // ------------------------------------------------------------ row statistics
         const int q = warp & 3;
         const int hcol = (warp - 4) >> 2;
@@ -211,20 +223,26 @@ __global__ void __launch_bounds__(384, 1)
             } else if (J == p.T - 1) {
                 jlim = p.n - J * 128;
             }
+            // Read this thread's 64 columns of S_t and S_s at once and hand the
+            // TMEM buffer back before the exponentials.
+            float st0[32], ss0[32], st1[32], ss1[32];
+            __syncwarp();
+            ptx::tmem_ld32(lane_base + buf * 256 + hcol * 64, st0);
+            ptx::tmem_ld32(lane_base + buf * 256 + 128 + hcol * 64, ss0);
+            ptx::tmem_ld32(lane_base + buf * 256 + hcol * 64 + 32, st1);
+            ptx::tmem_ld32(lane_base + buf * 256 + 128 + hcol * 64 + 32, ss1);
+            ptx::tmem_ld_wait(st0);
+            ptx::reg_dep(ss0);
+            ptx::reg_dep(st1);
+            ptx::reg_dep(ss1);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[buf]);
 #pragma unroll
             for (int round = 0; round < 2; ++round) {
                 const int cb = hcol * 64 + round * 32;
-                float st[32], ss[32];
-                __syncwarp();
-                ptx::tmem_ld32(lane_base + buf * 256 + cb, st);
-                ptx::tmem_ld32(lane_base + buf * 256 + 128 + cb, ss);
-                ptx::tmem_ld_wait(st);
-                ptx::reg_dep(ss);
-                if (round == 1) {
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[buf]);
-                }
+                float* st = round ? st1 : st0;
+                float* ss = round ? ss1 : ss0;
                 if (cb < jlim) {
                     if (cb + 32 > jlim) {
 #pragma unroll

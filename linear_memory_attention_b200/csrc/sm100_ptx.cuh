@@ -222,6 +222,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Warpgroup-wide register reallocation.  The shares of all warpgroups must
+// add up to (at most) the block's launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ----------------------------------------------------------------- misc
 __device__ __forceinline__ float ex2(float x) {
     float y;
