@@ -103,8 +103,8 @@ lard_status setup_device(int dev) {
         if (!ok) st = LARD_ERR_CUDA;
     }
     if (st == LARD_OK) {
-        const bool fits = split_fits(lard::lard_fwd_tc_kernel<64>, 384, lard::kFwdRegsSplitTotal) &&
-                          split_fits(lard::lard_fwd_tc_kernel<128>, 384, lard::kFwdRegsSplitTotal) &&
+        const bool fits = split_fits(lard::lard_fwd_tc_kernel<64>, lard::kFwdThreads, lard::kFwdRegsSplitTotal) &&
+                          split_fits(lard::lard_fwd_tc_kernel<128>, lard::kFwdThreads, lard::kFwdRegsSplitTotal) &&
                           split_fits(lard::lard_bwd_tc_kernel<64>, 512, lard::kBwdRegsSplitTotal) &&
                           split_fits(lard::lard_bwd_tc_kernel<128>, 512, lard::kBwdRegsSplitTotal);
         if (!fits) st = LARD_ERR_UNSUPPORTED;  // a build whose register count cannot host the split
@@ -238,10 +238,8 @@ lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const vo
 
     const int T = (n + 127) / 128;
     if (dtype == LARD_DTYPE_BF16) {
-        CUtensorMap mxt, myt, mxs, mys;
-        if (!make_map(&mxt, Xt, BH, n, d) || !make_map(&myt, Yt, BH, n, d) || !make_map(&mxs, Xs, BH, n, d) ||
-            !make_map(&mys, Ys, BH, n, d))
-            return LARD_ERR_INVALID_ARG;
+        CUtensorMap myt, mys;
+        if (!make_map(&myt, Yt, BH, n, d) || !make_map(&mys, Ys, BH, n, d)) return LARD_ERR_INVALID_ARG;
         lard::TcFwdParams p;
         p.BH = static_cast<int>(BH);
         p.n = n;
@@ -249,15 +247,17 @@ lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const vo
         p.causal = causal;
         p.tau = tau;
         p.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
+        p.Xt = static_cast<const __nv_bfloat16*>(Xt);
+        p.Xs = static_cast<const __nv_bfloat16*>(Xs);
         p.lse_t = lse_t;
         p.lse_s = lse_s;
         p.row_kl = row_kl;
         p.wait_ns = kWaitLimitNs;
         const unsigned grid = static_cast<unsigned>(BH * T);
         if (d == 128)
-            lard::lard_fwd_tc_kernel<128><<<grid, 384, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+            lard::lard_fwd_tc_kernel<128><<<grid, lard::kFwdThreads, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(myt, mys, p);
         else
-            lard::lard_fwd_tc_kernel<64><<<grid, 384, lard::FwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, p);
+            lard::lard_fwd_tc_kernel<64><<<grid, lard::kFwdThreads, lard::FwdLayout<64>::SMEM_BYTES, stream>>>(myt, mys, p);
     } else {
         lard::Fp32Params p;
         p.BH = static_cast<int>(BH);

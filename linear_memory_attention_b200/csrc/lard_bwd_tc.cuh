@@ -25,6 +25,7 @@
 //   warps 12-15  dX drain (TMEM -> smem -> TMA reduce-add), final dY store
 #pragma once
 
+#include "lard_exp2.cuh"
 #include "lard_kernel_common.cuh"
 
 namespace lard {
@@ -302,6 +303,7 @@ __global__ void __launch_bounds__(512, 1)
             else if (p.causal) { if (I == J) jlim = r + 1; }
             else if (J == p.T - 1) jlim = p.n - J * 128;
 
+            const float2 cf2 = splat2(cf), nbt2 = splat2(-bt), nbs2 = splat2(-bs), dzs2 = splat2(dzs);
             bool ok = ptx::mbar_wait(&ctrl->s_full, k & 1, abort_flag, lim, &g_lard_fault, kFaultBwdSoftmax);
             if (!__all_sync(0xffffffffu, ok)) break;
             ptx::tc_fence_after();
@@ -326,15 +328,19 @@ __global__ void __launch_bounds__(512, 1)
                 const float* st = round ? st1 : st0;
                 const float* ss = round ? ss1 : ss0;
                 uint32_t pk[16];
+                const bool masked = cb + 32 > jlim;  // only diagonal and tail tiles
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float rt0 = ptx::ex2(fmaf(st[c], cf, -bt));
-                    const float rs0 = ptx::ex2(fmaf(ss[c], cf, -bs));
-                    const float rt1 = ptx::ex2(fmaf(st[c + 1], cf, -bt));
-                    const float rs1 = ptx::ex2(fmaf(ss[c + 1], cf, -bs));
-                    const float d0 = (cb + c < jlim) ? (rs0 - rt0) * dzs : 0.f;
-                    const float d1 = (cb + c + 1 < jlim) ? (rs1 - rt1) * dzs : 0.f;
-                    pk[c >> 1] = ptx::pack_bf16x2(d0, d1);
+                    const float2 ut = fma2(make_float2(st[c], st[c + 1]), cf2, nbt2);
+                    const float2 us = fma2(make_float2(ss[c], ss[c + 1]), cf2, nbs2);
+                    const float2 rt = make_float2(ptx::ex2(ut.x), ptx::ex2(ut.y));
+                    const float2 rs = make_float2(ptx::ex2(us.x), ptx::ex2(us.y));
+                    float2 d = mul2(sub2(rs, rt), dzs2);
+                    if (masked) {
+                        if (cb + c >= jlim) d.x = 0.f;
+                        if (cb + c + 1 >= jlim) d.y = 0.f;
+                    }
+                    pk[c >> 1] = ptx::pack_bf16x2(d.x, d.y);
                 }
                 if (round == 0) {  // the dZ tile of k-1 must have been consumed by GEMMs 3 and 4
                     ok = ptx::mbar_wait(&ctrl->dz_free, (k & 1) ^ 1, abort_flag, lim, &g_lard_fault,
