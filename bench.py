@@ -12,7 +12,6 @@ batch (weak scaling); the relations of different ranks share nothing, so the
 timed region holds no collective.  Rank 0 prints one JSON line.
 """
 import argparse
-import dataclasses
 import json
 import math
 import os
@@ -169,16 +168,13 @@ def run_lard(args):
     import torch.distributed as dist
     from linear_memory_attention_b200 import lard, synth
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from linear_memory_attention_b200 import dist as ldist
+
+    rank, world, local = ldist.env_ranks()
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    ldist.init("nccl", device=torch.device("cuda", local))
     w = synth.WORKLOADS[args.workload]
-    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank)  # each rank: its own batch
+    wr = ldist.rank_workload(w, rank)  # each rank: its own batch
     host = synth.make_all(wr)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
@@ -239,12 +235,9 @@ def run_lard(args):
     elapsed_ms = t_start.elapsed_time(t_end)
     fwd_ms = {r: [e[r][0].elapsed_time(e[r][1]) for e in evs] for r in w.relations}
     bwd_ms = {r: [e[r][1].elapsed_time(e[r][2]) for e in evs] for r in w.relations}
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = ldist.max_over_ranks(elapsed_ms, device=dev)
     logits_step = w.causal_logits()
-    value = logits_step * K * world / (elapsed_ms / 1e3)
+    value = ldist.aggregate_rate(logits_step, K, world, elapsed_ms)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -274,12 +267,8 @@ def run_lard(args):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": logits_step * K * world / (e2e_ms / 1e3), "unit": UNIT,
+        e2e_ms = ldist.max_over_ranks(a.elapsed_time(b), device=dev)
+        e2e = {"value": ldist.aggregate_rate(logits_step, K, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / K}
 

@@ -125,6 +125,17 @@ LARD_API const char* lard_status_string(lard_status s);
  */
 LARD_API lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits);
 
+/*
+ * Failure-detection self-test: enqueues one small kernel whose single wait
+ * (an mbarrier that nothing arrives at) runs out after `limit_us`
+ * microseconds (1 .. 5e6).  The kernel then sets its bit (0x8000) in the
+ * device fault word and returns normally, so that a following
+ * lard_device_status() reports LARD_ERR_TIMEOUT with that bit while the
+ * CUDA context stays usable.  The pages define no counterpart; this checks
+ * the bounded waits every kernel of this library relies on.
+ */
+LARD_API lard_status lard_selftest_timeout(unsigned int limit_us, cudaStream_t stream);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 LARD_API int lard_version(void);
 

@@ -359,6 +359,16 @@ lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits) {
     return LARD_OK;
 }
 
+lard_status lard_selftest_timeout(unsigned int limit_us, cudaStream_t stream) {
+    if (limit_us == 0 || limit_us > 5000000u) return LARD_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LARD_ERR_CUDA;
+    lard_status st = setup_device(dev);
+    if (st != LARD_OK) return st;
+    lard::lard_selftest_timeout_kernel<<<1, 32, 0, stream>>>(1000ull * limit_us);
+    return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
+}
+
 int lard_version(void) { return kVersion; }
 
 }  // extern "C"

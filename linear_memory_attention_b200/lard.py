@@ -26,7 +26,8 @@ LIB_PATH = os.path.join(HERE, "liblard.so")
 LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT = range(5)
 LARD_DTYPE_BF16, LARD_DTYPE_FP32 = 0, 1
 
-EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status", "lard_version")
+EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status",
+           "lard_selftest_timeout", "lard_version")
 
 
 class LardError(RuntimeError):
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
     lib.lard_status_string.argtypes = [i]
     lib.lard_device_status.restype = i
     lib.lard_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.lard_selftest_timeout.restype = i
+    lib.lard_selftest_timeout.argtypes = [ctypes.c_uint, vp]
     lib.lard_version.restype = i
     lib.lard_version.argtypes = []
     return lib
@@ -133,6 +136,13 @@ def lard_device_status(stream=None) -> int:
         err.fault_bits = bits.value
         raise err
     return bits.value
+
+
+def lard_selftest_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test kernel (its wait runs out after limit_us)."""
+    st = _lib.lard_selftest_timeout(int(limit_us), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_selftest_timeout")
 
 
 def relation_kl(Xt, Xs, tau, causal=True, Yt=None, Ys=None, grad_scale=1.0, backward=True,
