@@ -284,7 +284,7 @@ def run_lard(args):
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     step_tflops = w.algorithmic_flops() * K / (elapsed_ms / 1e3) / 1e12  # per rank
-    traffic = _profiled_traffic(dom, w)
+    traffic, traffic_basis = _profiled_traffic(f"lard_{dom}_tc_kernel<{d}>", w)
 
     if rank == 0:
         out = {
@@ -303,7 +303,8 @@ def run_lard(args):
             "roofline": {"kernel": f"lard_{dom}_tc_kernel<{d}>", "bound": "tensor",
                          "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                          "peak_kind": f"bf16 dense, sustained ({peak_src})",
-                         "frac_of_burst_peak": ach / burst, "traffic": traffic},
+                         "frac_of_burst_peak": ach / burst, "traffic": traffic,
+                         "traffic_basis": traffic_basis},
             "kernel_ms": {"fwd": {r: statistics.mean(v) for r, v in fwd_ms.items()},
                           "bwd": {r: statistics.mean(v) for r, v in bwd_ms.items()}},
             "clocks": clk,
@@ -323,8 +324,9 @@ def run_lard(args):
 
 
 def _profiled_traffic(kernel, w):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary
-    for this workload, if one exists and matches the current kernel build."""
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary for this workload, if one exists and was taken on the current
+    kernel sources (else None: the counters no longer describe this kernel)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -332,10 +334,10 @@ def _profiled_traffic(kernel, w):
         ent = tab[f"{kernel}:{w.name}"]
         from linear_memory_attention_b200 import build
         if ent.get("source_digest") != build.source_digest():
-            return None
-        return ent["bytes_per_launch"]
+            return None, "kernel changed since the counters were taken"
+        return ent["bytes_per_launch"], ent.get("basis")
     except (OSError, ValueError, KeyError, AttributeError):
-        return None
+        return None, "no capture for this kernel and workload"
 
 
 def main():
