@@ -248,12 +248,27 @@ def run_lard(args):
                   for xt, xs in pinned.values())
         d2h = loss_host.numel() * loss_host.element_size()
 
+        # Each relation has its own device input buffers: its host->device copy
+        # runs on a copy stream as soon as that relation's previous compute has
+        # released them, so the copies of later relations overlap the kernels
+        # of earlier ones.  Every step still moves all its inputs and losses.
+        copy_stream = torch.cuda.Stream(device=dev)
+        released = {r: mk() for r in w.relations}
+        copied = {r: mk() for r in w.relations}
+        for r in w.relations:
+            released[r].record(stream)
+
         def e2e_step():
+            for r in w.relations:
+                copy_stream.wait_event(released[r])
+                with torch.cuda.stream(copy_stream):
+                    X[r][0].copy_(pinned[r][0], non_blocking=True)
+                    X[r][1].copy_(pinned[r][1], non_blocking=True)
+                copied[r].record(copy_stream)
             for idx, r in enumerate(w.relations):
-                xt, xs = X[r]
-                xt.copy_(pinned[r][0], non_blocking=True)
-                xs.copy_(pinned[r][1], non_blocking=True)
-                relation(r, xt, xs)
+                stream.wait_event(copied[r])
+                relation(r, *X[r])
+                released[r].record(stream)
                 loss_host[idx:idx + 1].copy_(O[r]["loss"], non_blocking=True)
 
         for _ in range(min(2, args.warmup)):
@@ -262,6 +277,7 @@ def run_lard(args):
         torch.cuda.synchronize()
         a, b = mk(), mk()
         a.record(stream)
+        copy_stream.wait_event(a)  # no copy of the timed steps starts before the region opens
         for _ in range(K):
             e2e_step()
         b.record(stream)

@@ -186,26 +186,33 @@ __global__ void __launch_bounds__(512, 1)
         constexpr uint32_t kIdescS = ptx::idesc_bf16(128, 128, 0, 0);
         constexpr uint32_t kIdescDY = ptx::idesc_bf16(128, D, 1, 1);
         constexpr uint32_t kIdescDX = ptx::idesc_bf16(128, D, 0, 1);
-        const uint32_t syt = ptx::smem_u32(smem + L::OFF_YT);
-        const uint32_t sys = ptx::smem_u32(smem + L::OFF_YS);
-        const uint32_t sxt = ptx::smem_u32(smem + L::OFF_XT);
-        const uint32_t sdz = ptx::smem_u32(smem + L::OFF_DZ);
-        auto sxs = [&](int k) { return ptx::smem_u32(smem + L::OFF_XS + (k & 1) * L::TILE); };
+        constexpr uint32_t kHi = ptx::sdesc_hi(1024);
+        // Descriptor low words, fixed for the CTA's life: K-major (leading offset
+        // 16 B) for the logit GEMMs and dZ as GEMM 4's A; MN-major (leading offset
+        // = one 64-column chunk) for dZ^T, X_s and Y_s in the gradient GEMMs.
+        const uint32_t yt_k = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_YT), 16);
+        const uint32_t ys_k = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_YS), 16);
+        const uint32_t ys_mn = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_YS), 16384);
+        const uint32_t xt_k = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_XT), 16);
+        const uint32_t xs_k0 = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_XS), 16);
+        const uint32_t xs_mn0 = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_XS), 16384);
+        const uint32_t dz_k = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_DZ), 16);
+        const uint32_t dz_mn = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_DZ), 16384);
+        constexpr uint32_t kStage = L::TILE >> 4;  // one X_s stage, in descriptor units
+        const uint32_t t_ss = tmem + kTmemSs, t_st = tmem + kTmemSt, t_dy = tmem + kTmemDY, t_dx = tmem + kTmemDX;
         auto issue_ss = [&](int k) {
-            const uint32_t a = sxs(k);
+            const uint32_t a = xs_k0 + (k & 1) * kStage;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                ptx::umma_bf16(tmem + kTmemSs, ptx::sdesc_sw128(a + koff, 16, 1024),
-                               ptx::sdesc_sw128(sys + koff, 16, 1024), kIdescS, kk > 0);
+                if (kk == 0) ptx::umma_ss<0>(t_ss, a, ys_k, kHi, kIdescS);
+                else ptx::umma_ss<1>(t_ss, a + ptx::desc_step_k(kk), ys_k + ptx::desc_step_k(kk), kHi, kIdescS);
             }
         };
         auto issue_st = [&]() {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                ptx::umma_bf16(tmem + kTmemSt, ptx::sdesc_sw128(sxt + koff, 16, 1024),
-                               ptx::sdesc_sw128(syt + koff, 16, 1024), kIdescS, kk > 0);
+                if (kk == 0) ptx::umma_ss<0>(t_st, xt_k, yt_k, kHi, kIdescS);
+                else ptx::umma_ss<1>(t_st, xt_k + ptx::desc_step_k(kk), yt_k + ptx::desc_step_k(kk), kHi, kIdescS);
             }
             ptx::umma_commit(&ctrl->xt_empty);
             ptx::umma_commit(&ctrl->s_full);
@@ -244,20 +251,18 @@ __global__ void __launch_bounds__(512, 1)
             if (!__all_sync(0xffffffffu, ok)) break;
             ptx::tc_fence_after();
             if (lane == 0) {
-                const uint32_t b3 = sxs(k);
+                const uint32_t b3 = xs_mn0 + (k & 1) * kStage;
                 // GEMM 3: dY[J] (+)= dZ^T X_s[I]; K runs over the 128 rows i, 16 per step.
+                ptx::umma_ss_acc(t_dy, dz_mn, b3, kHi, kIdescDY, k > 0 ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    ptx::umma_bf16(tmem + kTmemDY, ptx::sdesc_sw128(sdz + kk * 2048, 16384, 1024),
-                                   ptx::sdesc_sw128(b3 + kk * 2048, 16384, 1024), kIdescDY,
-                                   (k > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 1; kk < 8; ++kk)
+                    ptx::umma_ss<1>(t_dy, dz_mn + ptx::desc_step_mn(kk), b3 + ptx::desc_step_mn(kk), kHi, kIdescDY);
                 // GEMM 4: dX[I] = dZ Y_s[J]; K runs over the 128 columns j.
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    ptx::umma_bf16(tmem + kTmemDX,
-                                   ptx::sdesc_sw128(sdz + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                   ptx::sdesc_sw128(sys + kk * 2048, 16384, 1024), kIdescDX,
-                                   kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 8; ++kk) {
+                    if (kk == 0) ptx::umma_ss<0>(t_dx, dz_k, ys_mn, kHi, kIdescDX);
+                    else ptx::umma_ss<1>(t_dx, dz_k + ptx::desc_step_k(kk), ys_mn + ptx::desc_step_mn(kk), kHi, kIdescDX);
+                }
                 ptx::umma_commit(&ctrl->dz_free);
                 ptx::umma_commit(&ctrl->xs_empty[k & 1]);
                 ptx::umma_commit(&ctrl->dx_full);

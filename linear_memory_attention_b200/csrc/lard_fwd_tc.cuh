@@ -164,6 +164,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 128, 0, 0);
+        constexpr uint32_t kHi = ptx::sdesc_hi(1024);
+        // Descriptor low words of stage 0's Y_t; stage s and Y_s are fixed offsets.
+        const uint32_t y0_lo = ptx::sdesc_lo(ptx::smem_u32(smem + L::OFF_Y), 16);
+        const uint32_t st0 = tmem + kFwdTmemSt, ss = tmem + kFwdTmemSs;
+        const uint32_t xt = tmem + kFwdTmemXt, xs = tmem + kFwdTmemXs;
         bool ok = ptx::mbar_wait(&ctrl->x_ready, 0, abort_flag, lim, &g_lard_fault, kFaultFwdMma);
         ok = __all_sync(0xffffffffu, ok);
         for (int jt = 0; ok && jt < numJ; ++jt) {
@@ -174,15 +179,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                 kFaultFwdMma);
             if (!__all_sync(0xffffffffu, ok)) break;
             ptx::tc_fence_after();
-            const uint32_t syt = ptx::smem_u32(smem + L::OFF_Y + 2 * s * L::TILE);
-            const uint32_t sys = syt + L::TILE;
+            const uint32_t yt_lo = y0_lo + s * (2 * L::TILE >> 4);
+            const uint32_t ys_lo = yt_lo + (L::TILE >> 4);
             if (lane == 0) {
-                const uint32_t dt = tmem + kFwdTmemSt + buf * 128;
+                const uint32_t dt = st0 + buf * 128;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
-                    ptx::umma_bf16_ts(dt, tmem + kFwdTmemXt + k * 8, ptx::sdesc_sw128(syt + koff, 16, 1024),
-                                      kIdesc, k > 0);
+                    if (k == 0) ptx::umma_ts<0>(dt, xt, yt_lo, kHi, kIdesc);
+                    else ptx::umma_ts<1>(dt, xt + k * 8, yt_lo + ptx::desc_step_k(k), kHi, kIdesc);
                 }
             }
             __syncwarp();
@@ -193,9 +197,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (lane == 0) {
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
-                    ptx::umma_bf16_ts(tmem + kFwdTmemSs, tmem + kFwdTmemXs + k * 8,
-                                      ptx::sdesc_sw128(sys + koff, 16, 1024), kIdesc, k > 0);
+                    if (k == 0) ptx::umma_ts<0>(ss, xs, ys_lo, kHi, kIdesc);
+                    else ptx::umma_ts<1>(ss, xs + k * 8, ys_lo + ptx::desc_step_k(k), kHi, kIdesc);
                 }
                 ptx::umma_commit(&ctrl->y_empty[s]);
                 ptx::umma_commit(&ctrl->s_full[buf]);
@@ -312,9 +315,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     l_s *= ptx::ex2(m_s - nms);
                     m_s = nms;
                 }
-                // Column pairs in packed fp32x2 arithmetic; 5 of every 16 pairs
-                // take the FMA-pipe exponential so that the MUFU unit and the
-                // FMA pipe finish the tile together.
+                // Column pairs in packed fp32x2 arithmetic; 2 of every 16 pairs
+                // take the FMA-pipe exponential, which relieves the MUFU unit
+                // (16 exponentials per clock per SM).  More than that costs more
+                // than it saves: the polynomial takes 14 issue slots per pair
+                // against 2, and under the power cap the clock pays for them.
                 const float2 cf2 = splat2(cf), nmt2 = splat2(-m_t), nms2 = splat2(-m_s);
                 float2 LT = splat2(0.f), LS = splat2(0.f), AC = splat2(0.f);
 #pragma unroll
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const float2 ut = fma2(St, cf2, nmt2);
                     const float2 us = fma2(Ss, cf2, nms2);
                     const int pr = c >> 1;
-                    const bool on_fma = (pr == 1) || (pr == 4) || (pr == 7) || (pr == 10) || (pr == 13);
+                    const bool on_fma = (pr == 0) || (pr == 8);
                     const float2 pt = on_fma ? exp2_fma2(ut) : make_float2(ptx::ex2(ut.x), ptx::ex2(ut.y));
                     const float2 ps = on_fma ? exp2_fma2(us) : make_float2(ptx::ex2(us.x), ptx::ex2(us.y));
                     LT = add2(LT, pt);

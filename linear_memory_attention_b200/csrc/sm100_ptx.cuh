@@ -248,6 +248,64 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor as two 32-bit words, for issue loops that must stay
+// short: a single thread issues every MMA of the CTA, and at M = N = 128 the
+// tensor pipe finishes one K = 16 step in 64 cycles, so rebuilding 64-bit
+// descriptors per MMA makes the issuing thread, not the tensor pipe, the
+// bottleneck.  Shared-memory addresses of one CTA are below 2^18, so the
+// start-address field (bits 0-13) never carries into the leading offset and
+// the low word of the descriptor of (saddr + off) is sdesc_lo(saddr) + off/16.
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
+    return ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_hi(uint32_t sbo) {
+    return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+
+// Low-word advance of the descriptor for K step kk (16 bf16) of a tile stored as
+// 64-column chunks of 128-byte rows (16 KB per chunk of 128 rows):
+//   K-major operand:  chunk kk / 4, then 32 bytes per step inside the row;
+//   MN-major operand: 16 rows (2 KB) per step.
+__host__ __device__ constexpr uint32_t desc_step_k(int kk) { return (kk >> 2) * (16384 >> 4) + (kk & 3) * (32 >> 4); }
+__host__ __device__ constexpr uint32_t desc_step_mn(int kk) { return kk * (2048 >> 4); }
+
+// umma_bf16 / umma_bf16_ts with descriptor words and a compile-time
+// accumulate flag (ACC = 0: D = A B^T; 1: D += A B^T).
+template <uint32_t ACC>
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                        uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+__device__ __forceinline__ void umma_ss_acc(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 da, {%1, %3};\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+template <uint32_t ACC>
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                        uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "n"(ACC), "r"(idesc)
+        : "memory");
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn select MN-major (1) instead of K-major (0) operands.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
