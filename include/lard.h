@@ -106,13 +106,32 @@ LARD_API lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs,
  *                   dYs = g * dL/dYs = g * tau * dZ^T X_s,
  *                   with L = sum over (b, h) of the row-averaged KL.
  *                   They must not overlap each other or any input.
- * The bf16 path accumulates dXs with fp32 atomic adds, so its last bits
- * depend on the order in which tiles finish; the fp32 path is deterministic.
+ * The bf16 path accumulates dXs with fp32 reduce-adds in L2, so its last
+ * bits depend on the order in which tiles finish; the fp32 path is
+ * deterministic.
  */
 LARD_API lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys,
                         lard_dtype dtype, int B, int H, int n, int d, float tau, int causal,
                         const float* lse_t, const float* lse_s, float grad_scale,
                         float* dXs, float* dYs, cudaStream_t stream);
+
+/*
+ * Phase 2 for a self-relation (Y_t = X_t, Y_s = X_s, as for the Q/Q, K/K and
+ * V/V maps of LinearARD notes, 关键设计 1), returning the total student
+ * gradient: X_s enters the logits as both the row and the column factor, so
+ * dL/dX_s = tau dZ X_s + tau dZ^T X_s, the sum of lard_kl_bwd's dXs and dYs.
+ *
+ *   Xt, Xs, dtype, B, H, n, d, tau, causal, lse_t, lse_s, grad_scale: as for
+ *                   lard_kl_bwd with Yt = Xt and Ys = Xs.
+ *   dXs             out [B, H, n, d] fp32, overwritten with g * dL/dX_s (both
+ *                   paths); must not overlap any input.
+ * Both partials are added into dXs on the device (one n x d fp32 buffer and
+ * no separate sum).  LARD_ERR_UNSUPPORTED for fp32 inputs: call lard_kl_bwd
+ * and add dXs + dYs instead.
+ */
+LARD_API lard_status lard_kl_bwd_self(const void* Xt, const void* Xs, lard_dtype dtype, int B, int H, int n,
+                             int d, float tau, int causal, const float* lse_t, const float* lse_s,
+                             float grad_scale, float* dXs, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 LARD_API const char* lard_status_string(lard_status s);

@@ -274,24 +274,34 @@ lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const vo
     return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
 }
 
-lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
-                        int B, int H, int n, int d, float tau, int causal, const float* lse_t,
-                        const float* lse_s, float grad_scale, float* dXs, float* dYs, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Phase 2 for lard_kl_bwd (fuse = 0: dXs and dYs separately) and
+// lard_kl_bwd_self (fuse = 1: dYs == nullptr, both partials added into dXs).
+lard_status kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype, int B,
+                   int H, int n, int d, float tau, int causal, const float* lse_t, const float* lse_s,
+                   float grad_scale, float* dXs, float* dYs, int fuse, cudaStream_t stream) {
     long long BH = 0;
     lard_status st = check_common(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, &BH);
     if (st != LARD_OK) return st;
-    if (!lse_t || !lse_s || !dXs || !dYs) return LARD_ERR_INVALID_ARG;
+    if (!lse_t || !lse_s || !dXs || (!fuse && !dYs)) return LARD_ERR_INVALID_ARG;
     if (!std::isfinite(grad_scale)) return LARD_ERR_INVALID_ARG;
-    if (!aligned(lse_t, 4) || !aligned(lse_s, 4) || !aligned(dXs, 16) || !aligned(dYs, 16))
+    if (!aligned(lse_t, 4) || !aligned(lse_s, 4) || !aligned(dXs, 16) || (!fuse && !aligned(dYs, 16)))
         return LARD_ERR_INVALID_ARG;
     const size_t nin = in_bytes(dtype, BH, n, d), ngrad = static_cast<size_t>(BH) * n * d * 4;
     const size_t nrow = static_cast<size_t>(BH) * n * 4;
-    if (overlap(dXs, ngrad, dYs, ngrad)) return LARD_ERR_INVALID_ARG;
+    if (!fuse && overlap(dXs, ngrad, dYs, ngrad)) return LARD_ERR_INVALID_ARG;
     for (const void* g : {(const void*)dXs, (const void*)dYs}) {
+        if (!g) continue;
         for (const void* in : {Xt, Yt, Xs, Ys})
             if (overlap(g, ngrad, in, nin)) return LARD_ERR_INVALID_ARG;
         if (overlap(g, ngrad, lse_t, nrow) || overlap(g, ngrad, lse_s, nrow)) return LARD_ERR_INVALID_ARG;
     }
+    // The fp32 path parks per-row corrections in the dXs rows while it builds
+    // dYs, so it has no place to add dYs into dXs.
+    if (fuse && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
 
     DeviceGuard guard;
     st = select_device(Xt);
@@ -315,6 +325,7 @@ lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const vo
         p.lse_t = lse_t;
         p.lse_s = lse_s;
         p.dYs = dYs;
+        p.fuse_dy = fuse;
         p.wait_ns = kWaitLimitNs;
         const unsigned grid = static_cast<unsigned>(BH * T);
         if (d == 128)
@@ -333,6 +344,23 @@ lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const vo
                         stream);
     }
     return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
+                        int B, int H, int n, int d, float tau, int causal, const float* lse_t,
+                        const float* lse_s, float grad_scale, float* dXs, float* dYs, cudaStream_t stream) {
+    return kl_bwd(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, lse_t, lse_s, grad_scale, dXs, dYs, 0, stream);
+}
+
+lard_status lard_kl_bwd_self(const void* Xt, const void* Xs, lard_dtype dtype, int B, int H, int n, int d,
+                             float tau, int causal, const float* lse_t, const float* lse_s, float grad_scale,
+                             float* dXs, cudaStream_t stream) {
+    return kl_bwd(Xt, Xt, Xs, Xs, dtype, B, H, n, d, tau, causal, lse_t, lse_s, grad_scale, dXs, nullptr, 1,
+                  stream);
 }
 
 const char* lard_status_string(lard_status s) {

@@ -37,6 +37,7 @@ struct TcBwdParams {
     const float* lse_t;
     const float* lse_s;
     float* dYs;
+    int fuse_dy;  // 1: add dY_s into the dX_s buffer (self-relation total gradient), dYs unused
     unsigned long long wait_ns;
 };
 
@@ -373,6 +374,25 @@ __global__ void __launch_bounds__(512, 1)
         uint8_t* stage = smem + L::OFF_STG + q * 8192;  // this warp's two 4 KB boxes
         const uint32_t stage_u32 = ptx::smem_u32(stage);
         int nchunk = 0;
+        // Stage this warp's 32 x 32 box of fp32 values (one row per lane) in shared
+        // memory and add it into the gradient buffer at (column c * 32, row y0).
+        auto reduce_box = [&](const float (&v)[32], int c, int y0) {
+            const int b = nchunk & 1;
+            ++nchunk;
+            if (lane == 0) ptx::bulk_wait_read<1>();  // box b's previous reduce has read it
+            __syncwarp();
+            const uint32_t row = stage_u32 + b * 4096 + lane * 128;
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                ptx::st_shared_v4(row + ((u ^ (lane & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::tma_reduce_add_3d(&tm_dx, stage + b * 4096, c * 32, y0, bh);
+                ptx::bulk_commit();
+            }
+        };
         bool ok = true;
         for (int k = 0; k < K; ++k) {
             const int y0 = row_block(k) * 128 + q * 32;  // first dX row of this warp's box
@@ -390,28 +410,9 @@ __global__ void __launch_bounds__(512, 1)
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&ctrl->dx_free);
                 }
-                if (y0 < p.n) {  // warp-uniform: a box wholly past n is skipped
-                    const int b = nchunk & 1;
-                    ++nchunk;
-                    if (lane == 0) ptx::bulk_wait_read<1>();  // box b's previous reduce has read it
-                    __syncwarp();
-                    const uint32_t row = stage_u32 + b * 4096 + lane * 128;
-                    const uint32_t* w = reinterpret_cast<const uint32_t*>(v);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        ptx::st_shared_v4(row + ((u ^ (lane & 7)) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2],
-                                          w[4 * u + 3]);
-                    ptx::fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::tma_reduce_add_3d(&tm_dx, stage + b * 4096, c * 32, y0, bh);
-                        ptx::bulk_commit();
-                    }
-                }
+                if (y0 < p.n) reduce_box(v, c, y0);  // warp-uniform: a box wholly past n is skipped
             }
         }
-        if (lane == 0) ptx::bulk_wait<0>();
-        __syncwarp();
         if (ok) {
             ok = ptx::mbar_wait(&ctrl->dy_full, 0, abort_flag, lim, &g_lard_fault, kFaultBwdEpilogue);
             ok = __all_sync(0xffffffffu, ok);
@@ -419,14 +420,17 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) {
             ptx::tc_fence_after();
             const int j = J * 128 + r;
-            float* dst = p.dYs + (static_cast<size_t>(bh) * p.n + (j < p.n ? j : 0)) * D;
+            const int y0 = J * 128 + q * 32;
+            float* dst = p.fuse_dy ? nullptr : p.dYs + (static_cast<size_t>(bh) * p.n + (j < p.n ? j : 0)) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float v[32];
                 __syncwarp();
                 ptx::tmem_ld32(lane_base + kTmemDY + c * 32, v);
                 ptx::tmem_ld_wait(v);
-                if (j < p.n) {
+                if (p.fuse_dy) {
+                    if (y0 < p.n) reduce_box(v, c, y0);
+                } else if (j < p.n) {
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
                         *reinterpret_cast<float4*>(dst + c * 32 + 4 * u) =
@@ -434,6 +438,8 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
         }
+        if (lane == 0) ptx::bulk_wait<0>();
+        __syncwarp();
     }
 
     ptx::tc_fence_before();

@@ -10,6 +10,8 @@ Functions keep the C names:
                 loss_bh=None, loss_total=None, stream=None)
     lard_kl_bwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, grad_scale,
                 dXs, dYs, stream=None)
+    lard_kl_bwd_self(Xt, Xs, tau, causal, lse_t, lse_s, grad_scale, dXs,
+                     stream=None)
     lard_device_status(stream=None) -> fault bits (raises on timeout)
     lard_status_string(code), lard_version()
 Tensors are torch tensors [B, H, n, d] (inputs bf16 or fp32, outputs fp32),
@@ -26,8 +28,8 @@ LIB_PATH = os.path.join(HERE, "liblard.so")
 LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT = range(5)
 LARD_DTYPE_BF16, LARD_DTYPE_FP32 = 0, 1
 
-EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status",
-           "lard_selftest_timeout", "lard_version")
+EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_kl_bwd_self", "lard_status_string",
+           "lard_device_status", "lard_selftest_timeout", "lard_version")
 
 
 class LardError(RuntimeError):
@@ -47,6 +49,8 @@ def _load() -> ctypes.CDLL:
     lib.lard_kl_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, f32p, f32p, f32p, f32p, f32p, vp]
     lib.lard_kl_bwd.restype = i
     lib.lard_kl_bwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, f32p, f32p, f, f32p, f32p, vp]
+    lib.lard_kl_bwd_self.restype = i
+    lib.lard_kl_bwd_self.argtypes = [vp, vp, i, i, i, i, i, f, i, f32p, f32p, f, f32p, vp]
     lib.lard_status_string.restype = ctypes.c_char_p
     lib.lard_status_string.argtypes = [i]
     lib.lard_device_status.restype = i
@@ -125,6 +129,19 @@ def lard_kl_bwd(Xt, Yt, Xs, Ys, tau, causal, lse_t, lse_s, grad_scale, dXs, dYs,
                           _ptr(dXs), _ptr(dYs), _stream(stream))
     if st != LARD_OK:
         raise LardError(st, "lard_kl_bwd")
+
+
+def lard_kl_bwd_self(Xt, Xs, tau, causal, lse_t, lse_s, grad_scale, dXs, stream=None):
+    """Phase 2 of a self-relation: overwrites dXs [B,H,n,d] fp32 with grad_scale * dL/dXs
+    through both of Xs's roles (the sum of lard_kl_bwd's dXs and dYs).  bf16 inputs only."""
+    for t in (Xt, Xs):
+        if t.shape != Xt.shape or t.dtype != Xt.dtype or not t.is_contiguous():
+            raise ValueError("inputs must share one shape and dtype and be contiguous")
+    dt, B, H, n, d = _shape(Xt)
+    st = _lib.lard_kl_bwd_self(_ptr(Xt), _ptr(Xs), dt, B, H, n, d, float(tau), int(bool(causal)),
+                               _ptr(lse_t), _ptr(lse_s), float(grad_scale), _ptr(dXs), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_bwd_self")
 
 
 def lard_device_status(stream=None) -> int:

@@ -25,8 +25,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = declared_entry_points()
-    for n in ("lard_kl_fwd", "lard_kl_bwd", "lard_status_string", "lard_device_status",
-              "lard_version"):
+    for n in ("lard_kl_fwd", "lard_kl_bwd", "lard_kl_bwd_self", "lard_status_string",
+              "lard_device_status", "lard_selftest_timeout", "lard_version"):
         assert n in names
 
 
@@ -91,3 +91,17 @@ def test_fwd_rejects_bad_arguments(lib, kw, code):
 ])
 def test_bwd_rejects_bad_arguments(lib, kw, code):
     assert bwd(lib, **kw) == code
+
+
+def bwd_self(lib, *, dtype=0, n=300, d=128, tau=0.088, causal=1, g=1.0, dx=O3, lse_t=O1, lse_s=O2):
+    f = ctypes.c_float
+    return lib.lard_kl_bwd_self(A, C, dtype, 1, 2, n, d, f(tau), causal, lse_t, lse_s, f(g), dx, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dx=None), 1), (dict(lse_t=None), 1), (dict(g=float("nan")), 1), (dict(dx=A), 1),
+    (dict(dx=O1), 1), (dict(dx=O3 + 4), 1), (dict(d=32), 2), (dict(tau=0.0), 1),
+    (dict(dtype=1), 2),
+])
+def test_bwd_self_rejects_bad_arguments(lib, kw, code):
+    assert bwd_self(lib, **kw) == code
