@@ -210,10 +210,27 @@ def run_lard(args):
         if world > 1:
             dist.barrier()
 
+    # Device memory taken outside the caller's buffers: once on first use (the
+    # CUDA runtime loading the library's kernels), and per step after that (the
+    # library itself allocates nothing, so this should stay 0).
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info(dev)[0]
+    step()
+    torch.cuda.synchronize()
+    free2 = torch.cuda.mem_get_info(dev)[0]
     lard.lard_device_status()
+    # HBM state kept between the phases: LSE_t, LSE_s and row KL, 12 bytes per row.
+    rows_total = sum(w.B * w.heads[r] * n for r in w.relations)
+    extra_hbm = {"state_bytes": 12 * rows_total, "per_row_bytes": 12,
+                 "allocated_per_step_bytes": int(free1 - free2),
+                 "first_use_bytes": int(free0 - free1),
+                 "explicit_maps_bytes": 2 * 4 * sum(w.B * w.heads[r] * n * n for r in w.relations),
+                 "note": "state = lse_t, lse_s, row_kl (fp32, O(BHn)); explicit maps = the fp32 R_t and "
+                         "R_s that a materialising implementation would hold"}
 
     # ---------------------------------------------------------------- device-resident leg
     K = args.steps
@@ -325,6 +342,7 @@ def run_lard(args):
                           "bwd": {r: statistics.mean(v) for r, v in bwd_ms.items()}},
             "clocks": clk,
             "gpu_launches": 4 * len(w.relations) * K,
+            "extra_hbm": extra_hbm,
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:

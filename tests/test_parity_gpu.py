@@ -242,3 +242,18 @@ def test_workload_n32768(lard):
     w = synth.WORKLOADS["n32768"]
     _run_workload(lard, w, _check_rows(w, {r: [(0, 0), (0, 17)] for r in w.relations}, n_tail=160,
                                        n_random=16, seed=7))
+
+
+def test_long_single_head(lard):
+    """A long sequence (n = 131072 = 1024 row blocks, 5.4e5 causal tiles in one
+    head): tile coordinates far past the benchmark's, against the oracle on
+    tail rows (with the exact dY_s of the tail columns) and random rows."""
+    w = synth.custom(1, 1, 131072, 128, "bf16", seed=41, relations=("Q",))
+    _run_workload(lard, w, _check_rows(w, {"Q": [(0, 0)]}, n_tail=64, n_random=8, seed=8))
+
+
+def test_ragged_noncausal_whole_head(lard):
+    """No mask, n = 5000 (39 row blocks and a ragged 8-row tail), several heads:
+    the tail-column mask on every tile row; one whole head against the oracle."""
+    w = synth.custom(1, 3, 5000, 128, "bf16", seed=42, relations=("V",), causal=False)
+    _run_workload(lard, w, _check_heads(w, {"V": [(0, 2)]}))
