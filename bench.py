@@ -12,6 +12,7 @@ batch (weak scaling); the relations of different ranks share nothing, so the
 timed region holds no collective.  Rank 0 prints one JSON line.
 """
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -40,6 +41,8 @@ def parse_args():
                     help="one of: n32768 (default), n16384, n4096, gqa-n8000, fp32-small")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-mask", action="store_true",
+                    help="bidirectional relation maps (every logit allowed); metric then counts n*n logits")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time of the oracle sample")
     return ap.parse_args()
@@ -137,6 +140,10 @@ def run_reference(args):
         return
     from linear_memory_attention_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.no_mask:
+        w = dataclasses.replace(w, name=w.name + " no-mask", causal=False)
+    unit = UNIT if w.causal else "logits/s (no mask)"
+    metric = METRIC if w.causal else METRIC + " (no mask: every logit allowed)"
     host = synth.make_all(w)
     per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -152,14 +159,14 @@ def run_reference(args):
     sample = (f"per step: rows [n-{R}, n) of head (0,0) of each of {len(w.relations)} relations "
               f"({logits // max(1, args.steps)} causal logits), fp64 explicit maps")
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "B": w.B, "heads": w.heads, "n": w.n,
                                         "d": w.d, "causal": w.causal},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
@@ -174,6 +181,10 @@ def run_lard(args):
     torch.cuda.set_device(local)
     ldist.init("nccl", device=torch.device("cuda", local))
     w = synth.WORKLOADS[args.workload]
+    if args.no_mask:
+        w = dataclasses.replace(w, name=w.name + " no-mask", causal=False)
+    unit = UNIT if w.causal else "logits/s (no mask)"
+    metric = METRIC if w.causal else METRIC + " (no mask: every logit allowed)"
     wr = ldist.rank_workload(w, rank)  # each rank: its own batch
     host = synth.make_all(wr)
     dev = torch.device("cuda", local)
@@ -301,7 +312,7 @@ def run_lard(args):
         torch.cuda.synchronize()
         barrier()
         e2e_ms = ldist.max_over_ranks(a.elapsed_time(b), device=dev)
-        e2e = {"value": ldist.aggregate_rate(logits_step, K, world, e2e_ms), "unit": UNIT,
+        e2e = {"value": ldist.aggregate_rate(logits_step, K, world, e2e_ms), "unit": unit,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / K}
 
@@ -321,7 +332,7 @@ def run_lard(args):
 
     if rank == 0:
         out = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
             "data": "synthetic (seeded RoPE-shaped Q/K, Gaussian V; no weights or text)",
@@ -348,7 +359,7 @@ def run_lard(args):
         if world == 1 and not args.no_cpu_baseline:
             lg, dt, R, thr = oracle_sample(w, host, args.cpu_seconds)
             out["cpu_baseline"] = {
-                "value": lg / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+                "value": lg / dt, "unit": unit, "cores": thr, "kind": "oracle",
                 "sample": f"rows [n-{R}, n) of head (0,0) of each of {len(w.relations)} relations, "
                           f"{lg} causal logits in {dt:.1f} s, fp64 explicit maps"}
         print(json.dumps(out), flush=True)
