@@ -191,31 +191,35 @@ def run_lard(args):
     stream = torch.cuda.current_stream()
     f32 = dict(device=dev, dtype=torch.float32)
     B, n, d = w.B, w.n, w.d
-    X = {r: (xt.to(dev), xs.to(dev)) for r, (xt, xs) in host.items()}
+    R = len(w.relations)
+    # Two device copies of the inputs: the timed leg uses the first; the
+    # end-to-end leg alternates, so one step's host copies fill one set while
+    # the previous step computes on the other.
+    X = [{r: (xt.to(dev), xs.to(dev)) for r, (xt, xs) in host.items()} for _ in range(2)]
     O = {}
     for r in w.relations:
         H = w.heads[r]
         O[r] = dict(lse_t=torch.empty((B, H, n), **f32), lse_s=torch.empty((B, H, n), **f32),
-                    kl=torch.empty((B, H, n), **f32), loss_bh=torch.empty((B * H,), **f32),
-                    loss=torch.empty((1,), **f32), dX=torch.empty((B, H, n, d), **f32),
-                    dY=torch.empty((B, H, n, d), **f32))
+                    row_kl=torch.empty((B, H, n), **f32), loss_bh=torch.empty((B * H,), **f32),
+                    dXs=torch.empty((B, H, n, d), **f32), dYs=torch.empty((B, H, n, d), **f32))
+    loss = torch.empty((1,), **f32)  # the summed loss of the step's relations
+    rels = [[dict(Xt=X[k][r][0], Xs=X[k][r][1], **O[r]) for r in w.relations] for k in range(2)]
 
-    def relation(r, xt, xs, ev=None):
-        o = O[r]
+    def step(ev=None, k=0):
+        # One launch per phase for all relations (lard_kl_fwd_multi / _bwd_multi).
         if ev is not None:
             ev[0].record(stream)
-        lard.lard_kl_fwd(xt, xt, xs, xs, w.tau, w.causal, o["lse_t"], o["lse_s"], o["kl"],
-                         o["loss_bh"], o["loss"], stream)
+        lard.lard_kl_fwd_multi(rels[k], w.tau, w.causal, loss, stream)
         if ev is not None:
             ev[1].record(stream)
-        lard.lard_kl_bwd(xt, xt, xs, xs, w.tau, w.causal, o["lse_t"], o["lse_s"], 1.0, o["dX"],
-                         o["dY"], stream)
+        lard.lard_kl_bwd_multi(rels[k], w.tau, w.causal, 1.0, stream)
         if ev is not None:
             ev[2].record(stream)
 
-    def step(evs=None):
-        for r in w.relations:
-            relation(r, *X[r], None if evs is None else evs[r])
+    # Kernel launches per step: the bf16 path runs one Phase 1, one loss-rows,
+    # one loss-total and one Phase 2 kernel for all relations; the fp32 path
+    # runs Phase 1 per relation and three Phase 2 kernels per relation.
+    launches_per_step = 4 if w.dtype == "bf16" else R + 2 + 3 * R
 
     def barrier():
         if world > 1:
@@ -246,7 +250,7 @@ def run_lard(args):
     # ---------------------------------------------------------------- device-resident leg
     K = args.steps
     mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    evs = [{r: (mk(), mk(), mk()) for r in w.relations} for _ in range(K)]
+    evs = [(mk(), mk(), mk()) for _ in range(K)]
     clocks = ClockSampler(local)
     barrier()
     torch.cuda.synchronize()
@@ -261,8 +265,8 @@ def run_lard(args):
     barrier()
     lard.lard_device_status()
     elapsed_ms = t_start.elapsed_time(t_end)
-    fwd_ms = {r: [e[r][0].elapsed_time(e[r][1]) for e in evs] for r in w.relations}
-    bwd_ms = {r: [e[r][1].elapsed_time(e[r][2]) for e in evs] for r in w.relations}
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
     elapsed_ms = ldist.max_over_ranks(elapsed_ms, device=dev)
     logits_step = w.causal_logits()
     value = ldist.aggregate_rate(logits_step, K, world, elapsed_ms)
@@ -271,33 +275,35 @@ def run_lard(args):
     e2e = None
     if not args.no_e2e:
         pinned = {r: (xt.pin_memory(), xs.pin_memory()) for r, (xt, xs) in host.items()}
-        loss_host = torch.empty((len(w.relations),), dtype=torch.float32).pin_memory()
+        loss_host = torch.empty((1,), dtype=torch.float32).pin_memory()
         h2d = sum(xt.numel() * xt.element_size() + xs.numel() * xs.element_size()
                   for xt, xs in pinned.values())
         d2h = loss_host.numel() * loss_host.element_size()
 
-        # Each relation has its own device input buffers: its host->device copy
-        # runs on a copy stream as soon as that relation's previous compute has
-        # released them, so the copies of later relations overlap the kernels
-        # of earlier ones.  Every step still moves all its inputs and losses.
+        # Every step copies all its inputs from pinned host memory into one of
+        # the two device sets (on a copy stream, once the set's previous step has
+        # finished with it), runs both phases on that set, and reads the summed
+        # loss back.  So the copies of step k + 1 overlap the kernels of step k.
         copy_stream = torch.cuda.Stream(device=dev)
-        released = {r: mk() for r in w.relations}
-        copied = {r: mk() for r in w.relations}
-        for r in w.relations:
-            released[r].record(stream)
+        released = [mk(), mk()]
+        copied = [mk(), mk()]
+        for ev in released:
+            ev.record(stream)
+        counter = [0]
 
         def e2e_step():
-            for r in w.relations:
-                copy_stream.wait_event(released[r])
-                with torch.cuda.stream(copy_stream):
-                    X[r][0].copy_(pinned[r][0], non_blocking=True)
-                    X[r][1].copy_(pinned[r][1], non_blocking=True)
-                copied[r].record(copy_stream)
-            for idx, r in enumerate(w.relations):
-                stream.wait_event(copied[r])
-                relation(r, *X[r])
-                released[r].record(stream)
-                loss_host[idx:idx + 1].copy_(O[r]["loss"], non_blocking=True)
+            k = counter[0] % 2
+            counter[0] += 1
+            copy_stream.wait_event(released[k])
+            with torch.cuda.stream(copy_stream):
+                for r in w.relations:
+                    X[k][r][0].copy_(pinned[r][0], non_blocking=True)
+                    X[k][r][1].copy_(pinned[r][1], non_blocking=True)
+            copied[k].record(copy_stream)
+            stream.wait_event(copied[k])
+            step(k=k)
+            released[k].record(stream)
+            loss_host.copy_(loss, non_blocking=True)
 
         for _ in range(min(2, args.warmup)):
             e2e_step()
@@ -318,13 +324,11 @@ def run_lard(args):
 
     # ---------------------------------------------------------------- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
-    tot_f = sum(sum(v) for v in fwd_ms.values())
-    tot_b = sum(sum(v) for v in bwd_ms.values())
-    dom, dom_ms = ("bwd", bwd_ms) if tot_b >= tot_f else ("fwd", fwd_ms)
+    dom, dom_ms = ("bwd", bwd_ms) if sum(bwd_ms) >= sum(fwd_ms) else ("fwd", fwd_ms)
     gemms = 4 if dom == "bwd" else 2
-    per_launch_flops = {r: 2 * gemms * d * w.B * w.heads[r] *
-                        (n * (n + 1) // 2 if w.causal else n * n) for r in w.relations}
-    ach = statistics.mean(per_launch_flops[r] / (ms / 1e3) for r in w.relations for ms in dom_ms[r]) / 1e12
+    per_launch_flops = sum(2 * gemms * d * w.B * w.heads[r] * (n * (n + 1) // 2 if w.causal else n * n)
+                           for r in w.relations)
+    ach = statistics.mean(per_launch_flops / (ms / 1e3) for ms in dom_ms) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     step_tflops = w.algorithmic_flops() * K / (elapsed_ms / 1e3) / 1e12  # per rank
@@ -349,10 +353,10 @@ def run_lard(args):
                          "peak_kind": f"bf16 dense, sustained ({peak_src})",
                          "frac_of_burst_peak": ach / burst, "traffic": traffic,
                          "traffic_basis": traffic_basis},
-            "kernel_ms": {"fwd": {r: statistics.mean(v) for r, v in fwd_ms.items()},
-                          "bwd": {r: statistics.mean(v) for r, v in bwd_ms.items()}},
+            "kernel_ms": {"fwd": statistics.mean(fwd_ms), "bwd": statistics.mean(bwd_ms),
+                          "relations_per_launch": R if w.dtype == "bf16" else 1},
             "clocks": clk,
-            "gpu_launches": 4 * len(w.relations) * K,
+            "gpu_launches": launches_per_step * K,
             "extra_hbm": extra_hbm,
             "e2e": e2e,
         }

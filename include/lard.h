@@ -133,6 +133,59 @@ LARD_API lard_status lard_kl_bwd_self(const void* Xt, const void* Xs, lard_dtype
                              int d, float tau, int causal, const float* lse_t, const float* lse_s,
                              float grad_scale, float* dXs, cudaStream_t stream);
 
+/*
+ * Several relations in one launch per phase.  LinearARD distils three
+ * self-relations per layer (Q/Q, K/K, V/V; LinearARD notes, 关键设计 1), and a
+ * GQA model has fewer K/V heads than Q heads; one launch over all of them
+ * replaces a launch (and its tail) per relation.  Each relation is:
+ *
+ *   Xt, Yt, Xs, Ys  in [B, H, n, d] (as for lard_kl_fwd; Yt may equal Xt and
+ *                   Ys may equal Xs).
+ *   H               its head count (>= 1).
+ *   lse_t, lse_s    [B, H, n]: written by lard_kl_fwd_multi, read by
+ *                   lard_kl_bwd_multi.
+ *   row_kl          [B, H, n]: written by lard_kl_fwd_multi.
+ *   loss_bh         [B*H] or NULL: written by lard_kl_fwd_multi.
+ *   dXs             [B, H, n, d] fp32: written by lard_kl_bwd_multi.
+ *   dYs             [B, H, n, d] fp32, written by lard_kl_bwd_multi; or NULL
+ *                   for a self-relation (Yt == Xt, Ys == Xs, bf16 only), whose
+ *                   total student gradient is then written to dXs, as by
+ *                   lard_kl_bwd_self.
+ * Fields a phase does not use may be NULL.
+ */
+#define LARD_MAX_RELATIONS 4
+typedef struct lard_relation {
+    const void* Xt;
+    const void* Yt;
+    const void* Xs;
+    const void* Ys;
+    int H;
+    float* lse_t;
+    float* lse_s;
+    float* row_kl;
+    float* loss_bh;
+    float* dXs;
+    float* dYs;
+} lard_relation;
+
+/*
+ * Phase 1 of nrel (1 .. LARD_MAX_RELATIONS) relations sharing dtype, B, n, d,
+ * tau and causal.  Each relation's outputs are what lard_kl_fwd writes for
+ * it.  loss_total (or NULL; requires every loss_bh) is the sum of all
+ * relations' losses.  No output may overlap another buffer of the call; all
+ * buffers live on one GPU.  Errors as for lard_kl_fwd.
+ */
+LARD_API lard_status lard_kl_fwd_multi(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n,
+                              int d, float tau, int causal, float* loss_total, cudaStream_t stream);
+
+/*
+ * Phase 2 of nrel relations (as for lard_kl_fwd_multi, with the same inputs
+ * and the lse_t / lse_s it wrote).  Each relation's dXs (and dYs) are what
+ * lard_kl_bwd (or, with dYs == NULL, lard_kl_bwd_self) writes for it.
+ */
+LARD_API lard_status lard_kl_bwd_multi(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n,
+                              int d, float tau, int causal, float grad_scale, cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 LARD_API const char* lard_status_string(lard_status s);
 

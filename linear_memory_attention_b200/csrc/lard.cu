@@ -208,159 +208,287 @@ void launch_bwd_fp32(const float* Xt, const float* Yt, const float* Xs, const fl
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
-                        int B, int H, int n, int d, float tau, int causal, float* lse_t, float* lse_s,
-                        float* row_kl, float* loss_bh, float* loss_total, cudaStream_t stream) {
-    long long BH = 0;
-    lard_status st = check_common(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, &BH);
-    if (st != LARD_OK) return st;
-    if (!lse_t || !lse_s || !row_kl) return LARD_ERR_INVALID_ARG;
-    if (loss_total && !loss_bh) return LARD_ERR_INVALID_ARG;
-    for (const void* p : {(const void*)lse_t, (const void*)lse_s, (const void*)row_kl, (const void*)loss_bh,
-                          (const void*)loss_total})
-        if (p && !aligned(p, 4)) return LARD_ERR_INVALID_ARG;
-    const size_t nin = in_bytes(dtype, BH, n, d), nrow = static_cast<size_t>(BH) * n * 4;
-    const void* outs[5] = {lse_t, lse_s, row_kl, loss_bh, loss_total};
-    const size_t outn[5] = {nrow, nrow, nrow, static_cast<size_t>(BH) * 4, 4};
-    for (int a = 0; a < 5; ++a) {
-        if (!outs[a]) continue;
-        for (const void* in : {Xt, Yt, Xs, Ys})
-            if (overlap(outs[a], outn[a], in, nin)) return LARD_ERR_INVALID_ARG;
-        for (int b = a + 1; b < 5; ++b)
-            if (outs[b] && overlap(outs[a], outn[a], outs[b], outn[b])) return LARD_ERR_INVALID_ARG;
+// Byte ranges of one call's buffers: outputs may overlap nothing else.
+struct Ranges {
+    const void* p[64];
+    size_t n[64];
+    bool out[64];
+    int k = 0;
+    void add(const void* ptr, size_t bytes, bool is_out) {
+        if (!ptr || k >= 64) return;
+        p[k] = ptr;
+        n[k] = bytes;
+        out[k] = is_out;
+        ++k;
     }
+    bool outputs_disjoint() const {
+        for (int a = 0; a < k; ++a)
+            for (int b = a + 1; b < k; ++b)
+                if ((out[a] || out[b]) && overlap(p[a], n[a], p[b], n[b])) return false;
+        return true;
+    }
+};
+
+// Makes the GPU of the first relation current (and set up); every other
+// buffer must live on it.
+lard_status select_call_device(const lard_relation* rel, int nrel) {
+    lard_status st = select_device(rel[0].Xt);
+    if (st != LARD_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LARD_ERR_CUDA;
+    for (int r = 0; r < nrel; ++r)
+        for (const void* q : {rel[r].Xt, rel[r].Yt, rel[r].Xs, rel[r].Ys}) {
+            cudaPointerAttributes at;
+            if (cudaPointerGetAttributes(&at, q) != cudaSuccess) {
+                cudaGetLastError();
+                return LARD_ERR_INVALID_ARG;
+            }
+            if (at.device != dev) return LARD_ERR_INVALID_ARG;
+        }
+    return LARD_OK;
+}
+
+lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
+                   int causal, float* loss_total, cudaStream_t stream) {
+    if (!rel || nrel < 1 || nrel > lard::kMaxRelations) return LARD_ERR_INVALID_ARG;
+    long long BH[lard::kMaxRelations];
+    Ranges rg;
+    for (int r = 0; r < nrel; ++r) {
+        const lard_relation& R = rel[r];
+        lard_status st = check_common(R.Xt, R.Yt, R.Xs, R.Ys, dtype, B, R.H, n, d, tau, causal, &BH[r]);
+        if (st != LARD_OK) return st;
+        if (!R.lse_t || !R.lse_s || !R.row_kl) return LARD_ERR_INVALID_ARG;
+        if (loss_total && !R.loss_bh) return LARD_ERR_INVALID_ARG;
+        for (const void* q : {(const void*)R.lse_t, (const void*)R.lse_s, (const void*)R.row_kl,
+                              (const void*)R.loss_bh})
+            if (q && !aligned(q, 4)) return LARD_ERR_INVALID_ARG;
+        const size_t nin = in_bytes(dtype, BH[r], n, d), nrow = static_cast<size_t>(BH[r]) * n * 4;
+        for (const void* in : {R.Xt, R.Yt, R.Xs, R.Ys}) rg.add(in, nin, false);
+        rg.add(R.lse_t, nrow, true);
+        rg.add(R.lse_s, nrow, true);
+        rg.add(R.row_kl, nrow, true);
+        rg.add(R.loss_bh, static_cast<size_t>(BH[r]) * 4, true);
+    }
+    if (loss_total && !aligned(loss_total, 4)) return LARD_ERR_INVALID_ARG;
+    rg.add(loss_total, 4, true);
+    if (!rg.outputs_disjoint()) return LARD_ERR_INVALID_ARG;
 
     DeviceGuard guard;
-    st = select_device(Xt);
+    lard_status st = select_call_device(rel, nrel);
     if (st != LARD_OK) return st;
 
     const int T = (n + 127) / 128;
     if (dtype == LARD_DTYPE_BF16) {
-        CUtensorMap myt, mys;
-        if (!make_map(&myt, Yt, BH, n, d) || !make_map(&mys, Ys, BH, n, d)) return LARD_ERR_INVALID_ARG;
-        lard::TcFwdParams p;
-        p.BH = static_cast<int>(BH);
-        p.n = n;
-        p.T = T;
-        p.causal = causal;
-        p.tau = tau;
-        p.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
-        p.Xt = static_cast<const __nv_bfloat16*>(Xt);
-        p.Xs = static_cast<const __nv_bfloat16*>(Xs);
-        p.lse_t = lse_t;
-        p.lse_s = lse_s;
-        p.row_kl = row_kl;
-        p.wait_ns = kWaitLimitNs;
-        const unsigned grid = static_cast<unsigned>(BH * T);
+        lard::TcFwdGroup g;
+        long long blocks = 0;
+        for (int r = 0; r < nrel; ++r) {
+            if (!make_map(&g.yt[r], rel[r].Yt, BH[r], n, d) || !make_map(&g.ys[r], rel[r].Ys, BH[r], n, d))
+                return LARD_ERR_INVALID_ARG;
+            g.rel[r].Xt = static_cast<const __nv_bfloat16*>(rel[r].Xt);
+            g.rel[r].Xs = static_cast<const __nv_bfloat16*>(rel[r].Xs);
+            g.rel[r].lse_t = rel[r].lse_t;
+            g.rel[r].lse_s = rel[r].lse_s;
+            g.rel[r].row_kl = rel[r].row_kl;
+            g.rel[r].block0 = static_cast<int>(blocks);
+            blocks += BH[r] * T;
+        }
+        if (blocks > INT_MAX) return LARD_ERR_INVALID_ARG;
+        g.nrel = nrel;
+        g.n = n;
+        g.T = T;
+        g.causal = causal;
+        g.tau = tau;
+        g.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
+        g.wait_ns = kWaitLimitNs;
+        const unsigned grid = static_cast<unsigned>(blocks);
         if (d == 128)
-            lard::lard_fwd_tc_kernel<128><<<grid, lard::kFwdThreads, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(myt, mys, p);
+            lard::lard_fwd_tc_kernel<128><<<grid, lard::kFwdThreads, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(g);
         else
-            lard::lard_fwd_tc_kernel<64><<<grid, lard::kFwdThreads, lard::FwdLayout<64>::SMEM_BYTES, stream>>>(myt, mys, p);
+            lard::lard_fwd_tc_kernel<64><<<grid, lard::kFwdThreads, lard::FwdLayout<64>::SMEM_BYTES, stream>>>(g);
     } else {
-        lard::Fp32Params p;
-        p.BH = static_cast<int>(BH);
-        p.n = n;
-        p.causal = causal;
-        p.tau = tau;
-        p.dz_scale = 0.0;
-        LARD_DISPATCH_E(d, launch_fwd_fp32, static_cast<const float*>(Xt), static_cast<const float*>(Yt),
-                        static_cast<const float*>(Xs), static_cast<const float*>(Ys), p, lse_t, lse_s, row_kl,
-                        stream);
+        for (int r = 0; r < nrel; ++r) {
+            lard::Fp32Params p;
+            p.BH = static_cast<int>(BH[r]);
+            p.n = n;
+            p.causal = causal;
+            p.tau = tau;
+            p.dz_scale = 0.0;
+            LARD_DISPATCH_E(d, launch_fwd_fp32, static_cast<const float*>(rel[r].Xt),
+                            static_cast<const float*>(rel[r].Yt), static_cast<const float*>(rel[r].Xs),
+                            static_cast<const float*>(rel[r].Ys), p, rel[r].lse_t, rel[r].lse_s, rel[r].row_kl,
+                            stream);
+        }
     }
-    if (loss_bh) lard::lard_loss_rows_kernel<<<static_cast<unsigned>(BH), 256, 0, stream>>>(row_kl, n, loss_bh);
-    if (loss_total) lard::lard_loss_total_kernel<<<1, 256, 0, stream>>>(loss_bh, static_cast<int>(BH), loss_total);
+    // Per-head losses of every relation that asked for them, in one launch.
+    lard::LossRowsSet rows;
+    long long row_blocks = 0;
+    int k = 0;
+    for (int r = 0; r < nrel; ++r) {
+        if (!rel[r].loss_bh) continue;
+        rows.row_kl[k] = rel[r].row_kl;
+        rows.loss_bh[k] = rel[r].loss_bh;
+        rows.block0[k] = static_cast<int>(row_blocks);
+        row_blocks += BH[r];
+        ++k;
+    }
+    rows.nrel = k;
+    rows.n = n;
+    if (k > 0) lard::lard_loss_rows_kernel<<<static_cast<unsigned>(row_blocks), 256, 0, stream>>>(rows);
+    if (loss_total) {
+        lard::LossSet ls;
+        for (int r = 0; r < nrel; ++r) {
+            ls.loss_bh[r] = rel[r].loss_bh;
+            ls.BH[r] = static_cast<int>(BH[r]);
+        }
+        ls.nrel = nrel;
+        lard::lard_loss_total_kernel<<<1, 256, 0, stream>>>(ls, loss_total);
+    }
     return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
 }
 
-}  // extern "C"
-
-namespace {
-
-// Phase 2 for lard_kl_bwd (fuse = 0: dXs and dYs separately) and
-// lard_kl_bwd_self (fuse = 1: dYs == nullptr, both partials added into dXs).
-lard_status kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype, int B,
-                   int H, int n, int d, float tau, int causal, const float* lse_t, const float* lse_s,
-                   float grad_scale, float* dXs, float* dYs, int fuse, cudaStream_t stream) {
-    long long BH = 0;
-    lard_status st = check_common(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, &BH);
-    if (st != LARD_OK) return st;
-    if (!lse_t || !lse_s || !dXs || (!fuse && !dYs)) return LARD_ERR_INVALID_ARG;
+lard_status kl_bwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
+                   int causal, float grad_scale, cudaStream_t stream) {
+    if (!rel || nrel < 1 || nrel > lard::kMaxRelations) return LARD_ERR_INVALID_ARG;
     if (!std::isfinite(grad_scale)) return LARD_ERR_INVALID_ARG;
-    if (!aligned(lse_t, 4) || !aligned(lse_s, 4) || !aligned(dXs, 16) || (!fuse && !aligned(dYs, 16)))
-        return LARD_ERR_INVALID_ARG;
-    const size_t nin = in_bytes(dtype, BH, n, d), ngrad = static_cast<size_t>(BH) * n * d * 4;
-    const size_t nrow = static_cast<size_t>(BH) * n * 4;
-    if (!fuse && overlap(dXs, ngrad, dYs, ngrad)) return LARD_ERR_INVALID_ARG;
-    for (const void* g : {(const void*)dXs, (const void*)dYs}) {
-        if (!g) continue;
-        for (const void* in : {Xt, Yt, Xs, Ys})
-            if (overlap(g, ngrad, in, nin)) return LARD_ERR_INVALID_ARG;
-        if (overlap(g, ngrad, lse_t, nrow) || overlap(g, ngrad, lse_s, nrow)) return LARD_ERR_INVALID_ARG;
+    long long BH[lard::kMaxRelations];
+    Ranges rg;
+    bool fused_any = false;
+    for (int r = 0; r < nrel; ++r) {
+        const lard_relation& R = rel[r];
+        lard_status st = check_common(R.Xt, R.Yt, R.Xs, R.Ys, dtype, B, R.H, n, d, tau, causal, &BH[r]);
+        if (st != LARD_OK) return st;
+        if (!R.lse_t || !R.lse_s || !R.dXs) return LARD_ERR_INVALID_ARG;
+        const bool fuse = R.dYs == nullptr;
+        if (fuse && (R.Yt != R.Xt || R.Ys != R.Xs)) return LARD_ERR_INVALID_ARG;
+        fused_any = fused_any || fuse;
+        if (!aligned(R.lse_t, 4) || !aligned(R.lse_s, 4) || !aligned(R.dXs, 16) || (!fuse && !aligned(R.dYs, 16)))
+            return LARD_ERR_INVALID_ARG;
+        const size_t nin = in_bytes(dtype, BH[r], n, d), ngrad = static_cast<size_t>(BH[r]) * n * d * 4;
+        const size_t nrow = static_cast<size_t>(BH[r]) * n * 4;
+        for (const void* in : {R.Xt, R.Yt, R.Xs, R.Ys}) rg.add(in, nin, false);
+        rg.add(R.lse_t, nrow, false);
+        rg.add(R.lse_s, nrow, false);
+        rg.add(R.dXs, ngrad, true);
+        rg.add(R.dYs, ngrad, true);
     }
+    if (!rg.outputs_disjoint()) return LARD_ERR_INVALID_ARG;
     // The fp32 path parks per-row corrections in the dXs rows while it builds
     // dYs, so it has no place to add dYs into dXs.
-    if (fuse && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
+    if (fused_any && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
 
     DeviceGuard guard;
-    st = select_device(Xt);
+    lard_status st = select_call_device(rel, nrel);
     if (st != LARD_OK) return st;
 
     const int T = (n + 127) / 128;
     const double dz_scale = static_cast<double>(tau) * grad_scale / n;
     if (dtype == LARD_DTYPE_BF16) {
-        CUtensorMap mxt, myt, mxs, mys, mdx;
-        if (!make_map(&mxt, Xt, BH, n, d) || !make_map(&myt, Yt, BH, n, d) || !make_map(&mxs, Xs, BH, n, d) ||
-            !make_map(&mys, Ys, BH, n, d) || !make_grad_map(&mdx, dXs, BH, n, d))
-            return LARD_ERR_INVALID_ARG;
-        if (cudaMemsetAsync(dXs, 0, ngrad, stream) != cudaSuccess) return LARD_ERR_CUDA;
-        lard::TcBwdParams p;
-        p.BH = static_cast<int>(BH);
-        p.n = n;
-        p.T = T;
-        p.causal = causal;
-        p.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
-        p.dz_scale = static_cast<float>(dz_scale);
-        p.lse_t = lse_t;
-        p.lse_s = lse_s;
-        p.dYs = dYs;
-        p.fuse_dy = fuse;
-        p.wait_ns = kWaitLimitNs;
-        const unsigned grid = static_cast<unsigned>(BH * T);
+        lard::TcBwdGroup g;
+        long long blocks = 0;
+        for (int r = 0; r < nrel; ++r) {
+            const lard_relation& R = rel[r];
+            if (!make_map(&g.xt[r], R.Xt, BH[r], n, d) || !make_map(&g.yt[r], R.Yt, BH[r], n, d) ||
+                !make_map(&g.xs[r], R.Xs, BH[r], n, d) || !make_map(&g.ys[r], R.Ys, BH[r], n, d) ||
+                !make_grad_map(&g.dx[r], R.dXs, BH[r], n, d))
+                return LARD_ERR_INVALID_ARG;
+            g.rel[r].lse_t = R.lse_t;
+            g.rel[r].lse_s = R.lse_s;
+            g.rel[r].dYs = R.dYs;
+            g.rel[r].fuse_dy = R.dYs == nullptr;
+            g.rel[r].block0 = static_cast<int>(blocks);
+            blocks += BH[r] * T;
+        }
+        if (blocks > INT_MAX) return LARD_ERR_INVALID_ARG;
+        for (int r = 0; r < nrel; ++r)
+            if (cudaMemsetAsync(rel[r].dXs, 0, static_cast<size_t>(BH[r]) * n * d * 4, stream) != cudaSuccess)
+                return LARD_ERR_CUDA;
+        g.nrel = nrel;
+        g.n = n;
+        g.T = T;
+        g.causal = causal;
+        g.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
+        g.dz_scale = static_cast<float>(dz_scale);
+        g.wait_ns = kWaitLimitNs;
+        const unsigned grid = static_cast<unsigned>(blocks);
         if (d == 128)
-            lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, mdx, p);
+            lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(g);
         else
-            lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(mxt, myt, mxs, mys, mdx, p);
+            lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(g);
     } else {
-        lard::Fp32Params p;
-        p.BH = static_cast<int>(BH);
-        p.n = n;
-        p.causal = causal;
-        p.tau = tau;
-        p.dz_scale = dz_scale;
-        LARD_DISPATCH_E(d, launch_bwd_fp32, static_cast<const float*>(Xt), static_cast<const float*>(Yt),
-                        static_cast<const float*>(Xs), static_cast<const float*>(Ys), p, lse_t, lse_s, dXs, dYs,
-                        stream);
+        for (int r = 0; r < nrel; ++r) {
+            lard::Fp32Params p;
+            p.BH = static_cast<int>(BH[r]);
+            p.n = n;
+            p.causal = causal;
+            p.tau = tau;
+            p.dz_scale = dz_scale;
+            LARD_DISPATCH_E(d, launch_bwd_fp32, static_cast<const float*>(rel[r].Xt),
+                            static_cast<const float*>(rel[r].Yt), static_cast<const float*>(rel[r].Xs),
+                            static_cast<const float*>(rel[r].Ys), p, rel[r].lse_t, rel[r].lse_s, rel[r].dXs,
+                            rel[r].dYs, stream);
+        }
     }
     return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
+}
+
+lard_relation one_relation(const void* Xt, const void* Yt, const void* Xs, const void* Ys, int H) {
+    lard_relation R;
+    R.Xt = Xt;
+    R.Yt = Yt;
+    R.Xs = Xs;
+    R.Ys = Ys;
+    R.H = H;
+    R.lse_t = R.lse_s = R.row_kl = R.loss_bh = R.dXs = R.dYs = nullptr;
+    return R;
 }
 
 }  // namespace
 
 extern "C" {
 
+lard_status lard_kl_fwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
+                        int B, int H, int n, int d, float tau, int causal, float* lse_t, float* lse_s,
+                        float* row_kl, float* loss_bh, float* loss_total, cudaStream_t stream) {
+    lard_relation R = one_relation(Xt, Yt, Xs, Ys, H);
+    R.lse_t = lse_t;
+    R.lse_s = lse_s;
+    R.row_kl = row_kl;
+    R.loss_bh = loss_bh;
+    return kl_fwd(&R, 1, dtype, B, n, d, tau, causal, loss_total, stream);
+}
+
 lard_status lard_kl_bwd(const void* Xt, const void* Yt, const void* Xs, const void* Ys, lard_dtype dtype,
                         int B, int H, int n, int d, float tau, int causal, const float* lse_t,
                         const float* lse_s, float grad_scale, float* dXs, float* dYs, cudaStream_t stream) {
-    return kl_bwd(Xt, Yt, Xs, Ys, dtype, B, H, n, d, tau, causal, lse_t, lse_s, grad_scale, dXs, dYs, 0, stream);
+    if (!dYs) return LARD_ERR_INVALID_ARG;
+    lard_relation R = one_relation(Xt, Yt, Xs, Ys, H);
+    R.lse_t = const_cast<float*>(lse_t);
+    R.lse_s = const_cast<float*>(lse_s);
+    R.dXs = dXs;
+    R.dYs = dYs;
+    return kl_bwd(&R, 1, dtype, B, n, d, tau, causal, grad_scale, stream);
 }
 
 lard_status lard_kl_bwd_self(const void* Xt, const void* Xs, lard_dtype dtype, int B, int H, int n, int d,
                              float tau, int causal, const float* lse_t, const float* lse_s, float grad_scale,
                              float* dXs, cudaStream_t stream) {
-    return kl_bwd(Xt, Xt, Xs, Xs, dtype, B, H, n, d, tau, causal, lse_t, lse_s, grad_scale, dXs, nullptr, 1,
-                  stream);
+    lard_relation R = one_relation(Xt, Xt, Xs, Xs, H);
+    R.lse_t = const_cast<float*>(lse_t);
+    R.lse_s = const_cast<float*>(lse_s);
+    R.dXs = dXs;
+    return kl_bwd(&R, 1, dtype, B, n, d, tau, causal, grad_scale, stream);
+}
+
+lard_status lard_kl_fwd_multi(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d,
+                              float tau, int causal, float* loss_total, cudaStream_t stream) {
+    return kl_fwd(rel, nrel, dtype, B, n, d, tau, causal, loss_total, stream);
+}
+
+lard_status lard_kl_bwd_multi(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d,
+                              float tau, int causal, float grad_scale, cudaStream_t stream) {
+    return kl_bwd(rel, nrel, dtype, B, n, d, tau, causal, grad_scale, stream);
 }
 
 const char* lard_status_string(lard_status s) {

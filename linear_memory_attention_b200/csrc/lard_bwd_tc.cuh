@@ -30,14 +30,23 @@
 
 namespace lard {
 
-struct TcBwdParams {
-    int BH, n, T, causal;
-    float cfac;      // tau * log2(e)
-    float dz_scale;  // tau * grad_scale / n: dZ and the chain-rule tau in one factor
+// One relation of a launch.
+struct TcBwdRel {
     const float* lse_t;
     const float* lse_s;
     float* dYs;
     int fuse_dy;  // 1: add dY_s into the dX_s buffer (self-relation total gradient), dYs unused
+    int block0;   // first grid block of this relation (its B*H*T blocks follow)
+};
+
+// A launch: up to kMaxRelations relations of equal n and d in one grid.
+struct TcBwdGroup {
+    CUtensorMap xt[kMaxRelations], yt[kMaxRelations], xs[kMaxRelations], ys[kMaxRelations];
+    CUtensorMap dx[kMaxRelations];  // fp32 dX_s, for the reduce-adds
+    TcBwdRel rel[kMaxRelations];
+    int nrel, n, T, causal;
+    float cfac;      // tau * log2(e)
+    float dz_scale;  // tau * grad_scale / n: dZ and the chain-rule tau in one factor
     unsigned long long wait_ns;
 };
 
@@ -80,11 +89,7 @@ static_assert(kBwdRegsSplitTotal <= 512 * kBwdRegsLaunch, "register split exceed
 
 template <int D>
 __global__ void __launch_bounds__(512, 1)
-    lard_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_xt,
-                       const __grid_constant__ CUtensorMap tm_yt,
-                       const __grid_constant__ CUtensorMap tm_xs,
-                       const __grid_constant__ CUtensorMap tm_ys,
-                       const __grid_constant__ CUtensorMap tm_dx, const TcBwdParams p) {
+    lard_bwd_tc_kernel(const __grid_constant__ TcBwdGroup g) {
     using L = BwdLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -93,10 +98,27 @@ __global__ void __launch_bounds__(512, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Head-major order, longest column blocks first within a head: the blocks
-    // resident at any time then share one head's X tiles and dX rows in L2.
-    const int bh = static_cast<int>(blockIdx.x) / p.T;
-    const int J = static_cast<int>(blockIdx.x) % p.T;
+    // This block's relation; then head-major order within it, longest column
+    // blocks first within a head: the blocks resident at any time share one
+    // head's X tiles and dX rows in L2.
+    const int rel = relation_of_block(g.rel, g.nrel);
+    const CUtensorMap* tm_xt = &g.xt[rel];
+    const CUtensorMap* tm_yt = &g.yt[rel];
+    const CUtensorMap* tm_xs = &g.xs[rel];
+    const CUtensorMap* tm_ys = &g.ys[rel];
+    const CUtensorMap* tm_dx = &g.dx[rel];
+    const struct {
+        int n, T, causal;
+        float cfac, dz_scale;
+        const float *lse_t, *lse_s;
+        float* dYs;
+        int fuse_dy;
+        unsigned long long wait_ns;
+    } p = {g.n, g.T, g.causal, g.cfac, g.dz_scale, g.rel[rel].lse_t, g.rel[rel].lse_s, g.rel[rel].dYs,
+           g.rel[rel].fuse_dy, g.wait_ns};
+    const int local = static_cast<int>(blockIdx.x) - g.rel[rel].block0;
+    const int bh = local / p.T;
+    const int J = local % p.T;
     const int K = p.causal ? (p.T - J) : p.T;
     auto row_block = [&](int k) { return p.causal ? (J + k) : k; };
 
@@ -120,11 +142,11 @@ __global__ void __launch_bounds__(512, 1)
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tensormap(&tm_xt);
-        ptx::prefetch_tensormap(&tm_yt);
-        ptx::prefetch_tensormap(&tm_xs);
-        ptx::prefetch_tensormap(&tm_ys);
-        ptx::prefetch_tensormap(&tm_dx);
+        ptx::prefetch_tensormap(tm_xt);
+        ptx::prefetch_tensormap(tm_yt);
+        ptx::prefetch_tensormap(tm_xs);
+        ptx::prefetch_tensormap(tm_ys);
+        ptx::prefetch_tensormap(tm_dx);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&ctrl->tmem_base, 512);
@@ -142,8 +164,8 @@ __global__ void __launch_bounds__(512, 1)
         if (lane == 0) {
             ptx::mbar_arrive_expect_tx(&ctrl->y_full, 2 * L::TILE);
             for (int c = 0; c < L::KC; ++c) {
-                ptx::tma_load_3d(smem + L::OFF_YT + c * 16384, &tm_yt, &ctrl->y_full, c * 64, J * 128, bh);
-                ptx::tma_load_3d(smem + L::OFF_YS + c * 16384, &tm_ys, &ctrl->y_full, c * 64, J * 128, bh);
+                ptx::tma_load_3d(smem + L::OFF_YT + c * 16384, tm_yt, &ctrl->y_full, c * 64, J * 128, bh);
+                ptx::tma_load_3d(smem + L::OFF_YS + c * 16384, tm_ys, &ctrl->y_full, c * 64, J * 128, bh);
             }
         }
         __syncwarp();
@@ -157,7 +179,7 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) {
                 ptx::mbar_arrive_expect_tx(&ctrl->xt_full, L::TILE);
                 for (int c = 0; c < L::KC; ++c)
-                    ptx::tma_load_3d(smem + L::OFF_XT + c * 16384, &tm_xt, &ctrl->xt_full, c * 64, I * 128, bh);
+                    ptx::tma_load_3d(smem + L::OFF_XT + c * 16384, tm_xt, &ctrl->xt_full, c * 64, I * 128, bh);
             }
             __syncwarp();
             ++issued_t;
@@ -169,7 +191,7 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) {
                 ptx::mbar_arrive_expect_tx(&ctrl->xs_full[s], L::TILE);
                 for (int c = 0; c < L::KC; ++c)
-                    ptx::tma_load_3d(smem + L::OFF_XS + s * L::TILE + c * 16384, &tm_xs, &ctrl->xs_full[s],
+                    ptx::tma_load_3d(smem + L::OFF_XS + s * L::TILE + c * 16384, tm_xs, &ctrl->xs_full[s],
                                      c * 64, I * 128, bh);
             }
             __syncwarp();
@@ -389,7 +411,7 @@ __global__ void __launch_bounds__(512, 1)
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                ptx::tma_reduce_add_3d(&tm_dx, stage + b * 4096, c * 32, y0, bh);
+                ptx::tma_reduce_add_3d(tm_dx, stage + b * 4096, c * 32, y0, bh);
                 ptx::bulk_commit();
             }
         };

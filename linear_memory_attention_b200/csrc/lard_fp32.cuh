@@ -227,33 +227,56 @@ __global__ void __launch_bounds__(256) lard_bwd_dy_fp32_kernel(
     for (int e = 0; e < E; ++e) dYs[head + static_cast<size_t>(j) * D + lane + 32 * e] = static_cast<float>(acc[e]);
 }
 
-// loss_bh[bh] = (1/n) sum_i row_kl[bh, i]  (LinearARD notes, 关键设计 1: row-averaged KL).
-__global__ void __launch_bounds__(256) lard_loss_rows_kernel(const float* __restrict__ row_kl,
-                                                             int n, float* loss_bh) {
-    const int bh = blockIdx.x;
-    double s = 0.0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) s += row_kl[static_cast<size_t>(bh) * n + i];
+// Per-row KL arrays of the relations of one call, one grid block per (relation,
+// batch, head), relations one after the other.
+struct LossRowsSet {
+    const float* row_kl[kMaxRelations];
+    float* loss_bh[kMaxRelations];
+    int block0[kMaxRelations];  // first block of each relation
+    int nrel, n;
+};
+
+// loss_bh[bh] = (1/n) sum_i row_kl[bh, i] (LinearARD notes, 关键设计 1: the
+// row-averaged KL), summed in fp64.
+__global__ void __launch_bounds__(256) lard_loss_rows_kernel(const LossRowsSet s) {
+    int r = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int k = 1; k < kMaxRelations; ++k)
+        if (k < s.nrel && static_cast<int>(blockIdx.x) >= s.block0[k]) r = k;
+    const int bh = static_cast<int>(blockIdx.x) - s.block0[r];
+    const float* row_kl = s.row_kl[r];
+    const int n = s.n;
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) acc += row_kl[static_cast<size_t>(bh) * n + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     __shared__ double part[8];
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
     __syncthreads();
     if (threadIdx.x == 0) {
         double t = 0.0;
         for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += part[w];
-        loss_bh[bh] = static_cast<float>(t / n);
+        s.loss_bh[r][bh] = static_cast<float>(t / n);
     }
 }
 
-// loss_total = sum over (batch, head) of loss_bh.
-__global__ void __launch_bounds__(256) lard_loss_total_kernel(const float* __restrict__ loss_bh,
-                                                              int BH, float* loss_total) {
-    double s = 0.0;
-    for (int b = threadIdx.x; b < BH; b += blockDim.x) s += loss_bh[b];
+// Per-head losses of the relations of one call.
+struct LossSet {
+    const float* loss_bh[kMaxRelations];
+    int BH[kMaxRelations];
+    int nrel;
+};
+
+// loss_total = sum over relations and (batch, head) of loss_bh (the relations'
+// losses add with weight 1, LinearARD notes, 损失函数), summed in fp64.
+__global__ void __launch_bounds__(256) lard_loss_total_kernel(const LossSet s, float* loss_total) {
+    double acc = 0.0;
+    for (int r = 0; r < s.nrel; ++r)
+        for (int b = threadIdx.x; b < s.BH[r]; b += blockDim.x) acc += s.loss_bh[r][b];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     __shared__ double part[8];
-    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
     __syncthreads();
     if (threadIdx.x == 0) {
         double t = 0.0;

@@ -37,15 +37,25 @@
 
 namespace lard {
 
-struct TcFwdParams {
-    int BH, n, T, causal;
-    float cfac;  // tau * log2(e): S -> log2-domain logit
-    float tau;
+// One relation of a launch.
+struct TcFwdRel {
     const __nv_bfloat16* Xt;  // row sources of the TMEM-resident A operands
     const __nv_bfloat16* Xs;
     float* lse_t;
     float* lse_s;
     float* row_kl;
+    int block0;  // first grid block of this relation (its B*H*T blocks follow)
+};
+
+// A launch: up to kMaxRelations relations of equal n and d (for example the
+// Q/Q, K/K and V/V maps, with their own head counts) in one grid.
+struct TcFwdGroup {
+    CUtensorMap yt[kMaxRelations];  // Y_t and Y_s of each relation, {d, n, B*H}
+    CUtensorMap ys[kMaxRelations];
+    TcFwdRel rel[kMaxRelations];
+    int nrel, n, T, causal;
+    float cfac;  // tau * log2(e): S -> log2-domain logit
+    float tau;
     unsigned long long wait_ns;
 };
 
@@ -88,8 +98,7 @@ static_assert(sizeof(FwdCtrl) <= 8192, "control block too large");
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-    lard_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_yt, const __grid_constant__ CUtensorMap tm_ys,
-                       const TcFwdParams p) {
+    lard_fwd_tc_kernel(const __grid_constant__ TcFwdGroup g) {
     using L = FwdLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -98,10 +107,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Head-major order, longest row blocks first within a head: the blocks
-    // resident at any time then share one head's Y tiles, which stay in L2.
-    const int bh = static_cast<int>(blockIdx.x) / p.T;
-    const int I = p.T - 1 - static_cast<int>(blockIdx.x) % p.T;
+    // This block's relation; then head-major order within it, longest row
+    // blocks first within a head: the blocks resident at any time share one
+    // head's Y tiles, which stay in L2.
+    const int rel = relation_of_block(g.rel, g.nrel);
+    const CUtensorMap* tm_yt = &g.yt[rel];
+    const CUtensorMap* tm_ys = &g.ys[rel];
+    const struct {
+        int n, T, causal;
+        float cfac, tau;
+        const __nv_bfloat16 *Xt, *Xs;
+        float *lse_t, *lse_s, *row_kl;
+        unsigned long long wait_ns;
+    } p = {g.n, g.T, g.causal, g.cfac, g.tau, g.rel[rel].Xt, g.rel[rel].Xs, g.rel[rel].lse_t,
+           g.rel[rel].lse_s, g.rel[rel].row_kl, g.wait_ns};
+    const int local = static_cast<int>(blockIdx.x) - g.rel[rel].block0;
+    const int bh = local / p.T;
+    const int I = p.T - 1 - local % p.T;
     const int numJ = p.causal ? (I + 1) : p.T;
     auto col_block = [&](int jt) { return p.causal ? (I - jt) : ((I - jt + p.T) % p.T); };
 
@@ -121,8 +143,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::prefetch_tensormap(&tm_yt);
-        ptx::prefetch_tensormap(&tm_ys);
+        ptx::prefetch_tensormap(tm_yt);
+        ptx::prefetch_tensormap(tm_ys);
     }
     if (warp == 1) {
         ptx::tmem_alloc(&ctrl->tmem_base, 512);
@@ -149,8 +171,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 uint8_t* yt = smem + L::OFF_Y + 2 * s * L::TILE;
                 ptx::mbar_arrive_expect_tx(&ctrl->y_full[s], 2 * L::TILE);
                 for (int c = 0; c < L::KC; ++c) {
-                    ptx::tma_load_3d(yt + c * 16384, &tm_yt, &ctrl->y_full[s], c * 64, J * 128, bh);
-                    ptx::tma_load_3d(yt + L::TILE + c * 16384, &tm_ys, &ctrl->y_full[s], c * 64, J * 128, bh);
+                    ptx::tma_load_3d(yt + c * 16384, tm_yt, &ctrl->y_full[s], c * 64, J * 128, bh);
+                    ptx::tma_load_3d(yt + L::TILE + c * 16384, tm_ys, &ctrl->y_full[s], c * 64, J * 128, bh);
                 }
             }
             __syncwarp();

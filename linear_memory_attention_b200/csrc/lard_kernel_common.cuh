@@ -19,6 +19,21 @@ constexpr unsigned int kFaultBwdSoftmax = 1u << 6;
 constexpr unsigned int kFaultBwdEpilogue = 1u << 7;
 constexpr unsigned int kFaultSelfTest = 1u << 15;
 
+// Relations (X/Y pairs of equal n and d, any head counts) that one launch of a
+// tensor-core kernel may cover; their blocks are laid out one relation after
+// the other in the grid.
+constexpr int kMaxRelations = 4;
+
+// Relation of a grid block: the last r whose first block is <= blockIdx.x.
+template <typename Rel>
+__device__ __forceinline__ int relation_of_block(const Rel (&rel)[kMaxRelations], int nrel) {
+    int r = 0;
+#pragma unroll
+    for (int k = 1; k < kMaxRelations; ++k)
+        if (k < nrel && static_cast<int>(blockIdx.x) >= rel[k].block0) r = k;
+    return r;
+}
+
 // Exercises the bounded wait: one thread waits, with a short limit, on an
 // mbarrier that nothing arrives at; the wait runs out, raises the fault word
 // and the kernel returns normally.

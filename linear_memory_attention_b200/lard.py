@@ -12,6 +12,8 @@ Functions keep the C names:
                 dXs, dYs, stream=None)
     lard_kl_bwd_self(Xt, Xs, tau, causal, lse_t, lse_s, grad_scale, dXs,
                      stream=None)
+    lard_kl_fwd_multi(relations, tau, causal, loss_total=None, stream=None)
+    lard_kl_bwd_multi(relations, tau, causal, grad_scale, stream=None)
     lard_device_status(stream=None) -> fault bits (raises on timeout)
     lard_status_string(code), lard_version()
 Tensors are torch tensors [B, H, n, d] (inputs bf16 or fp32, outputs fp32),
@@ -28,8 +30,18 @@ LIB_PATH = os.path.join(HERE, "liblard.so")
 LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT = range(5)
 LARD_DTYPE_BF16, LARD_DTYPE_FP32 = 0, 1
 
-EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_kl_bwd_self", "lard_status_string",
-           "lard_device_status", "lard_selftest_timeout", "lard_version")
+EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_kl_bwd_self", "lard_kl_fwd_multi",
+           "lard_kl_bwd_multi", "lard_status_string", "lard_device_status", "lard_selftest_timeout",
+           "lard_version")
+LARD_MAX_RELATIONS = 4
+
+
+class _Relation(ctypes.Structure):
+    """struct lard_relation of include/lard.h."""
+    _fields_ = [("Xt", ctypes.c_void_p), ("Yt", ctypes.c_void_p), ("Xs", ctypes.c_void_p),
+                ("Ys", ctypes.c_void_p), ("H", ctypes.c_int), ("lse_t", ctypes.c_void_p),
+                ("lse_s", ctypes.c_void_p), ("row_kl", ctypes.c_void_p), ("loss_bh", ctypes.c_void_p),
+                ("dXs", ctypes.c_void_p), ("dYs", ctypes.c_void_p)]
 
 
 class LardError(RuntimeError):
@@ -51,6 +63,11 @@ def _load() -> ctypes.CDLL:
     lib.lard_kl_bwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, f32p, f32p, f, f32p, f32p, vp]
     lib.lard_kl_bwd_self.restype = i
     lib.lard_kl_bwd_self.argtypes = [vp, vp, i, i, i, i, i, f, i, f32p, f32p, f, f32p, vp]
+    rp = ctypes.POINTER(_Relation)
+    lib.lard_kl_fwd_multi.restype = i
+    lib.lard_kl_fwd_multi.argtypes = [rp, i, i, i, i, i, f, i, f32p, vp]
+    lib.lard_kl_bwd_multi.restype = i
+    lib.lard_kl_bwd_multi.argtypes = [rp, i, i, i, i, i, f, i, f, vp]
     lib.lard_status_string.restype = ctypes.c_char_p
     lib.lard_status_string.argtypes = [i]
     lib.lard_device_status.restype = i
@@ -142,6 +159,77 @@ def lard_kl_bwd_self(Xt, Xs, tau, causal, lse_t, lse_s, grad_scale, dXs, stream=
                                _ptr(lse_t), _ptr(lse_s), float(grad_scale), _ptr(dXs), _stream(stream))
     if st != LARD_OK:
         raise LardError(st, "lard_kl_bwd_self")
+
+
+def _relations(rels):
+    """ctypes array of lard_relation from dicts with the field names (tensors or None)."""
+    if not 1 <= len(rels) <= LARD_MAX_RELATIONS:
+        raise ValueError(f"1 to {LARD_MAX_RELATIONS} relations per call")
+    arr = (_Relation * len(rels))()
+    B = n = d = dt = None
+    for k, r in enumerate(rels):
+        Xt, Xs = r["Xt"], r["Xs"]
+        Yt, Ys = r.get("Yt", Xt), r.get("Ys", Xs)
+        _check_inputs(Xt, Yt, Xs, Ys)
+        dtk, Bk, Hk, nk, dk = _shape(Xt)
+        if B is None:
+            dt, B, n, d = dtk, Bk, nk, dk
+        elif (dtk, Bk, nk, dk) != (dt, B, n, d):
+            raise ValueError("relations of one call must share dtype, B, n and d")
+        arr[k].Xt, arr[k].Yt, arr[k].Xs, arr[k].Ys = (t.data_ptr() for t in (Xt, Yt, Xs, Ys))
+        arr[k].H = Hk
+        for name in ("lse_t", "lse_s", "row_kl", "loss_bh", "dXs", "dYs"):
+            t = r.get(name)
+            setattr(arr[k], name, None if t is None else t.data_ptr())
+    return arr, dt, B, n, d
+
+
+def lard_kl_fwd_multi(relations, tau, causal, loss_total=None, stream=None):
+    """Phase 1 of up to 4 relations in one launch.  ``relations``: dicts with Xt, Xs (and
+    optionally Yt, Ys; default Y = X), lse_t, lse_s, row_kl and optionally loss_bh."""
+    arr, dt, B, n, d = _relations(relations)
+    st = _lib.lard_kl_fwd_multi(arr, len(relations), dt, B, n, d, float(tau), int(bool(causal)),
+                                _ptr(loss_total), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_fwd_multi")
+
+
+def lard_kl_bwd_multi(relations, tau, causal, grad_scale, stream=None):
+    """Phase 2 of up to 4 relations in one launch.  ``relations``: dicts as for
+    lard_kl_fwd_multi with lse_t, lse_s, dXs and dYs; dYs None for a self-relation adds
+    both gradient paths into dXs."""
+    arr, dt, B, n, d = _relations(relations)
+    st = _lib.lard_kl_bwd_multi(arr, len(relations), dt, B, n, d, float(tau), int(bool(causal)),
+                                float(grad_scale), _stream(stream))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_bwd_multi")
+
+
+def relations_kl(pairs, tau, causal=True, grad_scale=1.0, backward=True, fused_self=False, stream=None):
+    """Both phases for several self-relations [(Xt, Xs), ...] in one launch per phase.
+
+    Returns (outputs per relation, loss): each output dict holds lse_t, lse_s, row_kl,
+    loss_bh and, if ``backward``, dXs (the total gradient if ``fused_self``) and dYs
+    (absent if ``fused_self``); loss is the summed loss of all relations (1 element).
+    """
+    import torch
+    outs, rels = [], []
+    for Xt, Xs in pairs:
+        B, H, n, d = Xt.shape
+        f32 = dict(device=Xt.device, dtype=torch.float32)
+        o = {"lse_t": torch.empty((B, H, n), **f32), "lse_s": torch.empty((B, H, n), **f32),
+             "row_kl": torch.empty((B, H, n), **f32), "loss_bh": torch.empty((B * H,), **f32)}
+        if backward:
+            o["dXs"] = torch.empty((B, H, n, d), **f32)
+            if not fused_self:
+                o["dYs"] = torch.empty((B, H, n, d), **f32)
+        outs.append(o)
+        rels.append(dict(Xt=Xt, Xs=Xs, **o))
+    loss = torch.empty((1,), device=pairs[0][0].device, dtype=torch.float32)
+    lard_kl_fwd_multi(rels, tau, causal, loss, stream)
+    if backward:
+        lard_kl_bwd_multi(rels, tau, causal, grad_scale, stream)
+    return outs, loss
 
 
 def lard_device_status(stream=None) -> int:

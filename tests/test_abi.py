@@ -105,3 +105,66 @@ def bwd_self(lib, *, dtype=0, n=300, d=128, tau=0.088, causal=1, g=1.0, dx=O3, l
 ])
 def test_bwd_self_rejects_bad_arguments(lib, kw, code):
     assert bwd_self(lib, **kw) == code
+
+
+def relations(specs):
+    from linear_memory_attention_b200.lard import _Relation
+    arr = (_Relation * max(1, len(specs)))()
+    for k, sp in enumerate(specs):
+        for name, v in sp.items():
+            setattr(arr[k], name, v)
+    return arr
+
+
+REL0 = dict(Xt=A, Yt=B_, Xs=C, Ys=D_, H=2, lse_t=O1, lse_s=O2, row_kl=O3, loss_bh=O4, dXs=O5,
+            dYs=0x1c000000)
+REL1 = dict(Xt=0x500000, Yt=0x500000, Xs=0x600000, Ys=0x600000, H=1, lse_t=0x15000000,
+            lse_s=0x16000000, row_kl=0x17000000, loss_bh=0x18000000, dXs=0x19000000, dYs=0x1a000000)
+
+
+def fwd_multi(lib, specs, nrel=None, dtype=0, n=300, d=128, loss=0x1b000000):
+    arr = relations(specs)
+    return lib.lard_kl_fwd_multi(arr, len(specs) if nrel is None else nrel, dtype, 1, n, d,
+                                 ctypes.c_float(0.088), 1, loss, None)
+
+
+def bwd_multi(lib, specs, nrel=None, dtype=0, n=300, d=128, g=1.0):
+    arr = relations(specs)
+    return lib.lard_kl_bwd_multi(arr, len(specs) if nrel is None else nrel, dtype, 1, n, d,
+                                 ctypes.c_float(0.088), 1, ctypes.c_float(g), None)
+
+
+@pytest.mark.parametrize("specs,nrel,code", [
+    ([REL0], 0, 1), ([REL0] * 5, 5, 1),
+    ([REL0, dict(REL1, row_kl=O3)], None, 1),          # two relations write one buffer
+    ([REL0, dict(REL1, lse_t=A)], None, 1),            # an output over another relation's input
+    ([REL0, dict(REL1, loss_bh=None)], None, 1),       # loss_total needs every loss_bh
+    ([REL0, dict(REL1, H=0)], None, 1),
+    ([REL0, dict(REL1, Xs=0x600008)], None, 1),        # misaligned input
+])
+def test_fwd_multi_rejects_bad_arguments(lib, specs, nrel, code):
+    assert fwd_multi(lib, specs, nrel) == code
+
+
+# A fused relation with fp32 inputs is refused (2) only after every range and
+# pointer check has passed, so a case that should fail those checks must give 1.
+FUSED1 = dict(REL1, dYs=None)
+
+
+def test_bwd_multi_valid_ranges_reach_the_dtype_check(lib):
+    assert bwd_multi(lib, [REL0, FUSED1], dtype=1) == 2
+
+
+@pytest.mark.parametrize("specs,kw,code", [
+    ([REL0, dict(FUSED1, dXs=O5)], {}, 1),             # two relations write one gradient
+    ([dict(REL0, dYs=0x600000), FUSED1], {}, 1),       # gradient over an input
+    ([dict(REL0, dYs=O1), FUSED1], {}, 1),             # gradient over an LSE input
+    ([dict(REL0, dYs=None), FUSED1], {}, 1),           # fused gradient needs Y = X
+    ([REL0, dict(FUSED1, lse_s=None)], {}, 1),
+    ([REL0, dict(FUSED1, dXs=0x19000004)], {}, 1),     # misaligned gradient
+    ([REL0, FUSED1], dict(g=float("inf")), 1),
+    ([REL0, FUSED1], dict(d=48), 2),                   # unsupported head size for fp32 (d % 32)
+])
+def test_bwd_multi_rejects_bad_arguments(lib, specs, kw, code):
+    kw = dict(dict(dtype=1), **kw)
+    assert bwd_multi(lib, specs, **kw) == code
