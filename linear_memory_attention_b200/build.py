@@ -25,10 +25,15 @@ def sources():
 
 
 def source_digest() -> str:
-    """Short hash of the kernel sources and header (identifies a kernel build)."""
+    """Short hash of the device code (the kernel headers, which also fix the
+    kernels' thread counts and shared-memory layouts): identifies the kernels
+    that a profile was taken of.  Host-side argument checks and the C ABI
+    wrappers in lard.cu do not enter it."""
     import hashlib
     h = hashlib.sha256()
     for path in sources():
+        if not path.endswith(".cuh"):
+            continue
         with open(path, "rb") as f:
             h.update(os.path.basename(path).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]

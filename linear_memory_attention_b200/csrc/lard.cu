@@ -232,21 +232,30 @@ struct Ranges {
 };
 
 // Makes the GPU of the first relation current (and set up); every other
-// buffer must live on it.
-lard_status select_call_device(const lard_relation* rel, int nrel) {
+// buffer of the call (`extra`, then each relation's fields) must be device or
+// managed memory on it.
+lard_status select_call_device(const lard_relation* rel, int nrel, const void* extra) {
     lard_status st = select_device(rel[0].Xt);
     if (st != LARD_OK) return st;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LARD_ERR_CUDA;
-    for (int r = 0; r < nrel; ++r)
-        for (const void* q : {rel[r].Xt, rel[r].Yt, rel[r].Xs, rel[r].Ys}) {
-            cudaPointerAttributes at;
-            if (cudaPointerGetAttributes(&at, q) != cudaSuccess) {
-                cudaGetLastError();
-                return LARD_ERR_INVALID_ARG;
-            }
-            if (at.device != dev) return LARD_ERR_INVALID_ARG;
+    auto on_dev = [&](const void* q) {
+        if (!q) return true;
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, q) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
         }
+        return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
+    };
+    if (!on_dev(extra)) return LARD_ERR_INVALID_ARG;
+    for (int r = 0; r < nrel; ++r) {
+        const lard_relation& R = rel[r];
+        for (const void* q : {R.Xt, R.Yt, R.Xs, R.Ys, (const void*)R.lse_t, (const void*)R.lse_s,
+                              (const void*)R.row_kl, (const void*)R.loss_bh, (const void*)R.dXs,
+                              (const void*)R.dYs})
+            if (!on_dev(q)) return LARD_ERR_INVALID_ARG;
+    }
     return LARD_OK;
 }
 
@@ -276,7 +285,7 @@ lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, 
     if (!rg.outputs_disjoint()) return LARD_ERR_INVALID_ARG;
 
     DeviceGuard guard;
-    lard_status st = select_call_device(rel, nrel);
+    lard_status st = select_call_device(rel, nrel, loss_total);
     if (st != LARD_OK) return st;
 
     const int T = (n + 127) / 128;
@@ -379,7 +388,7 @@ lard_status kl_bwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, 
     if (fused_any && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
 
     DeviceGuard guard;
-    lard_status st = select_call_device(rel, nrel);
+    lard_status st = select_call_device(rel, nrel, nullptr);
     if (st != LARD_OK) return st;
 
     const int T = (n + 127) / 128;
