@@ -6,11 +6,17 @@
 // contract it with the projections into dX_s and dY_s.  Fully masked tiles
 // (J > I) are never visited.
 //
-// One CTA owns a 128-column block J of one (batch, head); its dY_s[J]
+// One CTA owns a 128-column block J of one (batch, head) of one relation (a
+// launch covers up to kMaxRelations relations, TcBwdGroup); its dY_s[J]
 // accumulator stays in TMEM for the whole sweep over the row blocks I >= J
 // (all I without the mask).  Each tile's dX_s[I] contribution is staged in
 // shared memory and added to HBM with TMA bulk reduce-adds (fp32 adds in L2,
-// whole 128-byte lines, rows past n clipped by the tensor map).
+// whole 128-byte lines, rows past n clipped by the tensor map).  For a fused
+// self-relation the finished dY_s[J] is added into the same buffer the same
+// way; otherwise it is stored to dY_s.
+// The kernel is bound by shared-memory bandwidth: per tile the four SS GEMMs
+// read 256 KB of operands, and TMA writes, dZ stores and the dX staging add
+// another 224 KB; the GEMMs share the SM's shared-memory bandwidth with them.
 // TMEM (512 columns): dY [0, D), S_t [128, 256), S_s [256, 384), dX [384, 384 + D).
 // Shared memory: Y_t[J], Y_s[J] resident; a 2-stage ring for X_s[I]; one
 // buffer for X_t[I] (only the first GEMM of a tile reads it, so the next one
@@ -22,7 +28,7 @@
 // Roles (512 threads):
 //   warp 0       TMA producer          warp 1   TMEM owner, MMA issuer
 //   warps 4-11   dZ: one row per thread, one 64-column half per warpgroup
-//   warps 12-15  dX drain (TMEM -> smem -> TMA reduce-add), final dY store
+//   warps 12-15  dX drain (TMEM -> smem -> TMA reduce-add), final dY store or add
 #pragma once
 
 #include "lard_exp2.cuh"

@@ -6,8 +6,11 @@
 // This kernel also forms the row KL online from the same tiles (a
 // reading: the pages give no place for it; it needs no extra exponential).
 //
-// One CTA owns a 128-row block I of one (batch, head) and streams the column
-// blocks J it may attend to (J <= I under the causal mask), diagonal first.
+// One CTA owns a 128-row block I of one (batch, head) of one relation and
+// streams the column blocks J it may attend to (J <= I under the causal mask),
+// diagonal first.  A launch covers up to kMaxRelations relations (TcFwdGroup:
+// Q/Q, K/K and V/V with their own head counts); their blocks follow one
+// another in the grid.
 // X_t[I] and X_s[I] are the A operands of every GEMM of the CTA, so they are
 // kept in tensor memory (two bf16 per 32-bit column, row i in lane i): the
 // GEMMs then read only B = Y[J] from shared memory, which leaves shared-memory
