@@ -257,3 +257,11 @@ def test_ragged_noncausal_whole_head(lard):
     the tail-column mask on every tile row; one whole head against the oracle."""
     w = synth.custom(1, 3, 5000, 128, "bf16", seed=42, relations=("V",), causal=False)
     _run_workload(lard, w, _check_heads(w, {"V": [(0, 2)]}))
+
+
+@pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
+def test_head_dim_64_many_tiles(lard, causal):
+    """d = 64 (one 64-column chunk per tile row) over 24 row blocks with a ragged
+    tail, Q/Q and V/V, two heads; whole heads against the oracle."""
+    w = synth.custom(1, 2, 3000, 64, "bf16", seed=43, relations=("Q", "V"), causal=causal)
+    _run_workload(lard, w, _check_heads(w, {"Q": [(0, 1)], "V": [(0, 0)]}))
