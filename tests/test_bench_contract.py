@@ -1,0 +1,63 @@
+"""The benchmark's one-line JSON output: the fields and units a reader of the
+line relies on, for the reference arm (CPU) and the product arm (GPU)."""
+import json
+import math
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(args, timeout):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT,
+                         capture_output=True, text=True, timeout=timeout)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+COMMON = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+          "scaling", "vs_baseline", "dtype", "data", "config", "e2e", "cpu_baseline")
+
+
+def test_reference_arm_line():
+    d = _run(["--impl", "reference", "--workload", "n4096", "--steps", "1", "--warmup", "0"], 600)
+    for k in COMMON:
+        assert k in d, k
+    assert d["impl"] == "reference" and d["dtype"] == "f64" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["unit"] == "causal logits/s"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("qkv-self-relation") and d["config"]["n"] == 4096
+
+
+@pytest.mark.gpu
+def test_product_arm_line():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    K = 4
+    d = _run(["--workload", "n4096", "--steps", str(K), "--warmup", "3", "--cpu-seconds", "1"], 900)
+    for k in COMMON + ("roofline", "clocks", "gpu_launches", "extra_hbm", "tflops", "kernel_ms"):
+        assert k in d, k
+    assert d["n_gpus"] == 1 and d["steps"] == K and d["warmup"] == 3 and d["scaling"] == "weak"
+    assert d["dtype"] == "bf16" and d["vs_baseline"] is None and d["value"] > 0
+    r = d["roofline"]
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in r, k
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert 0 < r["frac"] < 1.5 and math.isclose(r["frac"], r["achieved"] / r["peak"], rel_tol=1e-9)
+    e = d["e2e"]
+    assert e["value"] > 0 and e["unit"] == d["unit"] and e["d2h_bytes_per_step"] == 4
+    assert e["h2d_bytes_per_step"] == 6 * 32 * 4096 * 128 * 2  # six bf16 input tensors per step
+    assert d["gpu_launches"] == 4 * K
+    assert d["extra_hbm"]["state_bytes"] == 12 * 3 * 32 * 4096
+    assert d["extra_hbm"]["allocated_per_step_bytes"] == 0
+    assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0 and cb["unit"] == d["unit"]
