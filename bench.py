@@ -333,6 +333,17 @@ def run_lard(args):
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     step_tflops = w.algorithmic_flops() * K / (elapsed_ms / 1e3) / 1e12  # per rank
     traffic, traffic_basis = _profiled_traffic(f"lard_{dom}_tc_kernel<{d}>", w)
+    # Phase 1 against the exponential unit: 2 exponentials per logit (teacher and
+    # student), MUFU at 16 per clock per SM on 148 SMs, at the median SM clock
+    # sampled during the timed region (a fraction of the polynomial share is on
+    # the FMA pipe, so the fraction can pass 1 in principle).
+    exps_per_launch = 2 * logits_step
+    mufu_peak = 16 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
+    mufu_ach = exps_per_launch / (statistics.mean(fwd_ms) / 1e3)
+    phase1_mufu = {"kernel": f"lard_fwd_tc_kernel<{d}>", "bound": "alu (MUFU exponentials)",
+                   "achieved": mufu_ach, "peak": mufu_peak, "unit": "exp2/s",
+                   "frac": (mufu_ach / mufu_peak) if mufu_peak else None,
+                   "peak_basis": "16 per clock per SM x 148 SMs x median sampled SM clock"}
 
     if rank == 0:
         out = {
@@ -353,6 +364,7 @@ def run_lard(args):
                          "peak_kind": f"bf16 dense, sustained ({peak_src})",
                          "frac_of_burst_peak": ach / burst, "traffic": traffic,
                          "traffic_basis": traffic_basis},
+            "phase1_roofline": phase1_mufu if w.dtype == "bf16" else None,
             "kernel_ms": {"fwd": statistics.mean(fwd_ms), "bwd": statistics.mean(bwd_ms),
                           "relations_per_launch": R if w.dtype == "bf16" else 1},
             "clocks": clk,
