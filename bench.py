@@ -340,6 +340,22 @@ def run_lard(args):
     exps_per_launch = 2 * logits_step
     mufu_peak = 16 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
     mufu_ach = exps_per_launch / (statistics.mean(fwd_ms) / 1e3)
+    # Phase 2 against shared-memory bandwidth, which binds it: per 128 x 128 tile
+    # the four SS GEMMs read 256 KB of operands (at d = 128), TMA writes 64 KB of
+    # X_t / X_s, the dZ warps store 32 KB, and the dX staging is written and read
+    # (128 KB); 128 bytes per clock per SM.
+    T = -(-n // 128)
+    tiles = sum(w.B * w.heads[r] for r in w.relations) * (T * (T + 1) // 2 if w.causal else T * T)
+    smem_per_tile = (256 + 64 + 32 + 128) * 1024 * d // 128
+    smem_peak = 128 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
+    smem_ach = tiles * smem_per_tile / (statistics.mean(bwd_ms) / 1e3)
+    phase2_smem = {"kernel": f"lard_bwd_tc_kernel<{d}>", "bound": "shared-memory bandwidth",
+                   "achieved": smem_ach / 1e9, "peak": smem_peak / 1e9 if smem_peak else None,
+                   "unit": "GB/s", "frac": (smem_ach / smem_peak) if smem_peak else None,
+                   "bytes_per_tile": smem_per_tile, "tiles_per_launch": tiles,
+                   "basis": "modelled bytes per 128x128 tile (MMA operand reads 256 KB, TMA writes 64 KB, "
+                            "dZ stores 32 KB, dX staging 128 KB at d = 128) over 128 B/clk/SM x 148 SMs "
+                            "x median sampled SM clock"}
     phase1_mufu = {"kernel": f"lard_fwd_tc_kernel<{d}>", "bound": "alu (MUFU exponentials)",
                    "achieved": mufu_ach, "peak": mufu_peak, "unit": "exp2/s",
                    "frac": (mufu_ach / mufu_peak) if mufu_peak else None,
@@ -365,6 +381,7 @@ def run_lard(args):
                          "frac_of_burst_peak": ach / burst, "traffic": traffic,
                          "traffic_basis": traffic_basis},
             "phase1_roofline": phase1_mufu if w.dtype == "bf16" else None,
+            "phase2_smem_roofline": phase2_smem if w.dtype == "bf16" else None,
             "kernel_ms": {"fwd": statistics.mean(fwd_ms), "bwd": statistics.mean(bwd_ms),
                           "relations_per_launch": R if w.dtype == "bf16" else 1},
             "clocks": clk,
