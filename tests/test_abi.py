@@ -168,3 +168,28 @@ def test_bwd_multi_valid_ranges_reach_the_dtype_check(lib):
 def test_bwd_multi_rejects_bad_arguments(lib, specs, kw, code):
     kw = dict(dict(dtype=1), **kw)
     assert bwd_multi(lib, specs, **kw) == code
+
+
+def test_binding_marshalling_errors():
+    """The Python binding's own checks, before any call into the library."""
+    import torch
+    from linear_memory_attention_b200 import lard
+    a = torch.zeros((1, 2, 64, 128), dtype=torch.bfloat16)
+    b = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16)
+    f = torch.zeros((1, 2, 64, 128), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        lard._relations([])                                   # no relation
+    with pytest.raises(ValueError):
+        lard._relations([dict(Xt=a, Xs=a)] * 5)               # more than LARD_MAX_RELATIONS
+    with pytest.raises(ValueError):
+        lard._relations([dict(Xt=a, Xs=a), dict(Xt=b, Xs=b)])  # relations of different d
+    with pytest.raises(ValueError):
+        lard._relations([dict(Xt=a, Xs=b)])                   # X_t and X_s of different shapes
+    with pytest.raises(ValueError):
+        lard._shape(f)                                        # unsupported dtype
+    with pytest.raises(ValueError):
+        lard._shape(a[0])                                     # not [B, H, n, d]
+    arr, dt, B, n, d = lard._relations([dict(Xt=a, Xs=a), dict(Xt=a[:, :1].contiguous(),
+                                                                Xs=a[:, :1].contiguous())])
+    assert (dt, B, n, d) == (lard.LARD_DTYPE_BF16, 1, 64, 128)
+    assert arr[0].H == 2 and arr[1].H == 1 and arr[0].Yt == arr[0].Xt and arr[1].dYs is None
