@@ -254,5 +254,30 @@ def pin_gibbs_rowsum_duality(orc):
         _close(o2["dXs"], np.zeros_like(Xs), 0.0, 1e-13 * max(scale, 1.0), "row sums (dX = 0)")
 
 
+def pin_self_relation_total_gradient(orc):
+    """A self-relation (Y = X, as Q/Q, K/K, V/V): torch autograd through one
+    tied student leaf gives the total gradient, which must be the sum of the
+    oracle's two partials dXs + dYs (the quantity lard_kl_bwd_self returns)."""
+    rng = _rng(17)
+    for causal in (True, False):
+        for (BH, n, d) in ((1, 5, 4), (2, 23, 8)):
+            tau = 1.0 / math.sqrt(d)
+            Xt, Xs = _rand(rng, BH, n, d, scale=1.3), _rand(rng, BH, n, d, scale=1.3)
+            o = orc.relation(Xt, Xt, Xs, Xs, tau, causal)
+            xt = torch.tensor(Xt)
+            xs = torch.tensor(Xs, requires_grad=True)
+            keep = torch.ones(n, n, dtype=torch.bool)
+            if causal:
+                keep = torch.tril(keep)
+            zt = (tau * xt @ xt.transpose(-1, -2)).masked_fill(~keep, -1e300)
+            zs = (tau * xs @ xs.transpose(-1, -2)).masked_fill(~keep, -1e300)
+            kl = torch.nn.functional.kl_div(torch.log_softmax(zs, -1), torch.log_softmax(zt, -1),
+                                            log_target=True, reduction="none").sum(-1)
+            kl.mean(-1).sum().backward()
+            _close(o["dXs"] + o["dYs"], xs.grad.numpy(), 1e-10, 1e-14,
+                   f"self-relation total gradient causal={causal} n={n}")
+
+
 PINS = [pin_finite_differences, pin_torch_autograd, pin_scipy_rows, pin_identical_student,
-        pin_causal_row0, pin_constant_rows, pin_binary_closed_form, pin_gibbs_rowsum_duality]
+        pin_causal_row0, pin_constant_rows, pin_binary_closed_form, pin_gibbs_rowsum_duality,
+        pin_self_relation_total_gradient]
