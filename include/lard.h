@@ -27,7 +27,9 @@
  *     entries are summed; a caller sums the three relations;
  *   - gradients carry the chain-rule factor tau of Z = tau X Y^T:
  *     dX_s = tau dZ Y_s, dY_s = tau dZ^T X_s; the teacher gets none;
- *   - for a self-relation (Y = X) the caller adds the two partials.
+ *   - for a self-relation (Y = X) the student gradient is the sum of the two
+ *     partials; lard_kl_bwd returns them apart, lard_kl_bwd_self (and
+ *     lard_kl_bwd_multi with dYs = NULL) adds them on the device.
  *
  * Conventions for every entry point:
  *   - Tensors are row-major [B, H, n, d], contiguous, in device memory of
