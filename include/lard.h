@@ -35,8 +35,9 @@
  *   - Tensors are row-major [B, H, n, d], contiguous, in device memory of
  *     the GPU that runs the call, base addresses 16-byte aligned.  Inputs
  *     are bf16 (LARD_DTYPE_BF16) or fp32 (LARD_DTYPE_FP32); every output is
- *     fp32.  The caller allocates and owns every buffer; the library
- *     allocates no device memory.
+ *     fp32, except the gradients of lard_kl_bwd_multi_bf16.  The caller
+ *     allocates and owns every buffer (and that call's workspace); the
+ *     library allocates no device memory.
  *   - Work is enqueued asynchronously on `stream` (0 = legacy default
  *     stream); results are valid once the stream reaches that point.
  *   - Argument errors are reported synchronously, before anything is
@@ -188,14 +189,65 @@ LARD_API lard_status lard_kl_fwd_multi(const lard_relation* rel, int nrel, lard_
 LARD_API lard_status lard_kl_bwd_multi(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n,
                               int d, float tau, int causal, float grad_scale, cudaStream_t stream);
 
+/*
+ * bf16 gradient outputs (Phase 2).  A bf16 training step consumes bf16
+ * gradients; writing them directly halves the gradient bytes the call writes
+ * and a caller copies out.  dY_s[J] is complete in the kernel and is rounded
+ * once; dX_s receives contributions from every column block of a row, so it
+ * is accumulated in fp32 in a caller-provided workspace and rounded once
+ * (round-to-nearest-even) by a final pass of the same call.  For a fused
+ * self-relation (dYs == NULL) both partials accumulate in the workspace and
+ * dXs receives the rounded total gradient.  This follows LinearARD notes,
+ * 关键设计 3 (gradients accumulated into dX_s and dY_s) with the rounding the
+ * pages leave open placed after the accumulation.
+ *
+ *   dXs, dYs   bf16 [B, H, n, d] outputs of one relation, 16-byte aligned;
+ *              dYs == NULL for a fused self-relation (Yt == Xt, Ys == Xs).
+ */
+typedef struct lard_grads_bf16 {
+    void* dXs;
+    void* dYs;
+} lard_grads_bf16;
+
+/*
+ * Bytes of fp32 workspace lard_kl_bwd_multi_bf16 needs for these relations:
+ * the sum over relations of B * H * n * d * 4.  Returns 0 if the description
+ * is invalid (rel NULL, nrel outside 1 .. LARD_MAX_RELATIONS, a size < 1).
+ */
+LARD_API size_t lard_kl_bwd_bf16_workspace_bytes(const lard_relation* rel, int nrel, int B, int n, int d);
+
+/*
+ * Phase 2 of nrel relations (as lard_kl_bwd_multi) with bf16 gradient outputs.
+ *   rel        as for lard_kl_bwd_multi, with every dXs and dYs field NULL (the
+ *              gradients go to `out`).
+ *   out        [nrel] bf16 output buffers, overwritten with what
+ *              lard_kl_bwd_multi writes in fp32, rounded once to bf16.
+ *   workspace  device memory on the call's GPU, 16-byte aligned, at least
+ *              lard_kl_bwd_bf16_workspace_bytes(rel, nrel, B, n, d) bytes
+ *              (workspace_bytes); its contents are overwritten and have no
+ *              meaning after the call; it must not overlap any other buffer.
+ * bf16 inputs only (LARD_ERR_UNSUPPORTED for fp32 inputs, whose path is the
+ * full-precision one).  Other errors as for lard_kl_bwd_multi.  The
+ * workspace is the only memory the call uses beyond its inputs and outputs;
+ * the library allocates none.
+ */
+LARD_API lard_status lard_kl_bwd_multi_bf16(const lard_relation* rel, const lard_grads_bf16* out, int nrel,
+                                   lard_dtype dtype, int B, int n, int d, float tau, int causal,
+                                   float grad_scale, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 LARD_API const char* lard_status_string(lard_status s);
 
 /*
  * Synchronises `stream`, then reads and clears the device-side fault word of
- * the current device.  Returns LARD_ERR_TIMEOUT if a kernel wait ran out of
+ * the GPU that `stream` belongs to (for the legacy default stream 0, the
+ * current device).  Returns LARD_ERR_TIMEOUT if a kernel wait ran out of
  * time since the last check (and stores the fault bits in *fault_bits if it
  * is not NULL), LARD_ERR_CUDA if synchronisation failed, else LARD_OK.
+ * Bits: 0x1-0x4 a Phase-1 role, 0x10-0x80 a Phase-2 role, 0x100 a block
+ * that left before its own copies or tensor-core work had finished (its
+ * exit wait ran out), 0x8000 the self-test below.
  */
 LARD_API lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits);
 

@@ -12,13 +12,15 @@
 #include "lard.h"
 #include "lard_kernel_common.cuh"
 #include "lard_bwd_tc.cuh"
+#include "lard_cast.cuh"
 #include "lard_fp32.cuh"
 #include "lard_fwd_tc.cuh"
 
 namespace {
 
-constexpr int kVersion = 100;                          // 0.1.0
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr int kVersion = 200;                          // 0.2.0
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long kDrainLimitNs = 8000000000ull;  // 8 s per drain on the way out
 constexpr int kMaxDevices = 64;
 constexpr long long kMaxElems = 1LL << 40;
 
@@ -234,7 +236,8 @@ struct Ranges {
 // Makes the GPU of the first relation current (and set up); every other
 // buffer of the call (`extra`, then each relation's fields) must be device or
 // managed memory on it.
-lard_status select_call_device(const lard_relation* rel, int nrel, const void* extra) {
+lard_status select_call_device(const lard_relation* rel, int nrel, const void* extra,
+                               const lard_grads_bf16* out16 = nullptr) {
     lard_status st = select_device(rel[0].Xt);
     if (st != LARD_OK) return st;
     int dev = 0;
@@ -255,8 +258,21 @@ lard_status select_call_device(const lard_relation* rel, int nrel, const void* e
                               (const void*)R.row_kl, (const void*)R.loss_bh, (const void*)R.dXs,
                               (const void*)R.dYs})
             if (!on_dev(q)) return LARD_ERR_INVALID_ARG;
+        if (out16 && (!on_dev(out16[r].dXs) || !on_dev(out16[r].dYs))) return LARD_ERR_INVALID_ARG;
     }
     return LARD_OK;
+}
+
+// Σ over relations of B * H * n * d * 4 bytes: the fp32 dX_s accumulators of a
+// Phase-2 call with bf16 outputs (0 for an invalid description).
+size_t bf16_workspace_bytes(const lard_relation* rel, int nrel, int B, int n, int d) {
+    if (!rel || nrel < 1 || nrel > lard::kMaxRelations || B < 1 || n < 1 || d < 1) return 0;
+    size_t total = 0;
+    for (int r = 0; r < nrel; ++r) {
+        if (rel[r].H < 1) return 0;
+        total += static_cast<size_t>(B) * rel[r].H * n * d * 4;
+    }
+    return total;
 }
 
 lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
@@ -311,6 +327,7 @@ lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, 
         g.tau = tau;
         g.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
         g.wait_ns = kWaitLimitNs;
+        g.drain_ns = kDrainLimitNs;
         const unsigned grid = static_cast<unsigned>(blocks);
         if (d == 128)
             lard::lard_fwd_tc_kernel<128><<<grid, lard::kFwdThreads, lard::FwdLayout<128>::SMEM_BYTES, stream>>>(g);
@@ -357,61 +374,96 @@ lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, 
     return cudaGetLastError() == cudaSuccess ? LARD_OK : LARD_ERR_CUDA;
 }
 
+// bf16 gradient outputs of a Phase-2 call: where they go and the fp32
+// workspace that accumulates dX_s (and, fused, dY_s) before the rounding.
+struct Bf16Grads {
+    const lard_grads_bf16* out;
+    void* ws;
+    size_t ws_bytes;
+};
+
 lard_status kl_bwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
-                   int causal, float grad_scale, cudaStream_t stream) {
+                   int causal, float grad_scale, cudaStream_t stream, const Bf16Grads* b16 = nullptr) {
     if (!rel || nrel < 1 || nrel > lard::kMaxRelations) return LARD_ERR_INVALID_ARG;
     if (!std::isfinite(grad_scale)) return LARD_ERR_INVALID_ARG;
+    if (b16 && !b16->out) return LARD_ERR_INVALID_ARG;
     long long BH[lard::kMaxRelations];
     Ranges rg;
     bool fused_any = false;
+    size_t ws_need = 0;
     for (int r = 0; r < nrel; ++r) {
         const lard_relation& R = rel[r];
         lard_status st = check_common(R.Xt, R.Yt, R.Xs, R.Ys, dtype, B, R.H, n, d, tau, causal, &BH[r]);
         if (st != LARD_OK) return st;
-        if (!R.lse_t || !R.lse_s || !R.dXs) return LARD_ERR_INVALID_ARG;
-        const bool fuse = R.dYs == nullptr;
+        if (!R.lse_t || !R.lse_s) return LARD_ERR_INVALID_ARG;
+        // The gradient buffers: fp32 in the relation, or bf16 in b16->out.
+        const void* gx = b16 ? b16->out[r].dXs : static_cast<const void*>(R.dXs);
+        const void* gy = b16 ? b16->out[r].dYs : static_cast<const void*>(R.dYs);
+        if (b16 && (R.dXs || R.dYs)) return LARD_ERR_INVALID_ARG;  // outputs are given once
+        if (!gx) return LARD_ERR_INVALID_ARG;
+        const bool fuse = gy == nullptr;
         if (fuse && (R.Yt != R.Xt || R.Ys != R.Xs)) return LARD_ERR_INVALID_ARG;
         fused_any = fused_any || fuse;
-        if (!aligned(R.lse_t, 4) || !aligned(R.lse_s, 4) || !aligned(R.dXs, 16) || (!fuse && !aligned(R.dYs, 16)))
+        if (!aligned(R.lse_t, 4) || !aligned(R.lse_s, 4) || !aligned(gx, 16) || (!fuse && !aligned(gy, 16)))
             return LARD_ERR_INVALID_ARG;
-        const size_t nin = in_bytes(dtype, BH[r], n, d), ngrad = static_cast<size_t>(BH[r]) * n * d * 4;
+        const size_t nin = in_bytes(dtype, BH[r], n, d);
+        const size_t ngrad = static_cast<size_t>(BH[r]) * n * d * (b16 ? 2 : 4);
         const size_t nrow = static_cast<size_t>(BH[r]) * n * 4;
         for (const void* in : {R.Xt, R.Yt, R.Xs, R.Ys}) rg.add(in, nin, false);
         rg.add(R.lse_t, nrow, false);
         rg.add(R.lse_s, nrow, false);
-        rg.add(R.dXs, ngrad, true);
-        rg.add(R.dYs, ngrad, true);
+        rg.add(gx, ngrad, true);
+        rg.add(gy, ngrad, true);
+        ws_need += static_cast<size_t>(BH[r]) * n * d * 4;
+    }
+    if (b16) {
+        if (!b16->ws || !aligned(b16->ws, 16) || b16->ws_bytes < ws_need) return LARD_ERR_INVALID_ARG;
+        rg.add(b16->ws, ws_need, true);
     }
     if (!rg.outputs_disjoint()) return LARD_ERR_INVALID_ARG;
     // The fp32 path parks per-row corrections in the dXs rows while it builds
-    // dYs, so it has no place to add dYs into dXs.
-    if (fused_any && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
+    // dYs, so it has no place to add dYs into dXs; and it is the full-precision
+    // path, which bf16 outputs would defeat.
+    if ((fused_any || b16) && dtype != LARD_DTYPE_BF16) return LARD_ERR_UNSUPPORTED;
 
     DeviceGuard guard;
-    lard_status st = select_call_device(rel, nrel, nullptr);
+    lard_status st = select_call_device(rel, nrel, b16 ? b16->ws : nullptr, b16 ? b16->out : nullptr);
     if (st != LARD_OK) return st;
 
     const int T = (n + 127) / 128;
     const double dz_scale = static_cast<double>(tau) * grad_scale / n;
     if (dtype == LARD_DTYPE_BF16) {
         lard::TcBwdGroup g;
+        lard::CastSet cast;
         long long blocks = 0;
+        float* acc[lard::kMaxRelations];  // fp32 dX_s accumulator of each relation
+        size_t ws_off = 0;
+        cast.start8[0] = 0;
         for (int r = 0; r < nrel; ++r) {
             const lard_relation& R = rel[r];
+            const size_t elems = static_cast<size_t>(BH[r]) * n * d;
+            acc[r] = b16 ? reinterpret_cast<float*>(static_cast<char*>(b16->ws) + ws_off) : R.dXs;
+            ws_off += elems * 4;
             if (!make_map(&g.xt[r], R.Xt, BH[r], n, d) || !make_map(&g.yt[r], R.Yt, BH[r], n, d) ||
                 !make_map(&g.xs[r], R.Xs, BH[r], n, d) || !make_map(&g.ys[r], R.Ys, BH[r], n, d) ||
-                !make_grad_map(&g.dx[r], R.dXs, BH[r], n, d))
+                !make_grad_map(&g.dx[r], acc[r], BH[r], n, d))
                 return LARD_ERR_INVALID_ARG;
             g.rel[r].lse_t = R.lse_t;
             g.rel[r].lse_s = R.lse_s;
-            g.rel[r].dYs = R.dYs;
-            g.rel[r].fuse_dy = R.dYs == nullptr;
+            g.rel[r].dYs = b16 ? nullptr : R.dYs;
+            g.rel[r].dYs_bf16 = b16 ? static_cast<__nv_bfloat16*>(b16->out[r].dYs) : nullptr;
+            g.rel[r].fuse_dy = (b16 ? b16->out[r].dYs : static_cast<void*>(R.dYs)) == nullptr;
             g.rel[r].block0 = static_cast<int>(blocks);
             blocks += BH[r] * T;
+            if (b16) {
+                cast.src[r] = acc[r];
+                cast.dst[r] = static_cast<__nv_bfloat16*>(b16->out[r].dXs);
+                cast.start8[r + 1] = cast.start8[r] + static_cast<long long>(elems / 8);
+            }
         }
         if (blocks > INT_MAX) return LARD_ERR_INVALID_ARG;
         for (int r = 0; r < nrel; ++r)
-            if (cudaMemsetAsync(rel[r].dXs, 0, static_cast<size_t>(BH[r]) * n * d * 4, stream) != cudaSuccess)
+            if (cudaMemsetAsync(acc[r], 0, static_cast<size_t>(BH[r]) * n * d * 4, stream) != cudaSuccess)
                 return LARD_ERR_CUDA;
         g.nrel = nrel;
         g.n = n;
@@ -420,11 +472,21 @@ lard_status kl_bwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, 
         g.cfac = static_cast<float>(static_cast<double>(tau) * 1.4426950408889634);
         g.dz_scale = static_cast<float>(dz_scale);
         g.wait_ns = kWaitLimitNs;
+        g.drain_ns = kDrainLimitNs;
         const unsigned grid = static_cast<unsigned>(blocks);
         if (d == 128)
             lard::lard_bwd_tc_kernel<128><<<grid, 512, lard::BwdLayout<128>::SMEM_BYTES, stream>>>(g);
         else
             lard::lard_bwd_tc_kernel<64><<<grid, 512, lard::BwdLayout<64>::SMEM_BYTES, stream>>>(g);
+        if (b16) {
+            cast.nrel = nrel;
+            int dev = 0, sms = 148;
+            if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            const long long groups = cast.start8[nrel];
+            const long long want = (groups + 255) / 256;
+            const unsigned cgrid = static_cast<unsigned>(want < 8LL * sms ? (want > 0 ? want : 1) : 8LL * sms);
+            lard::lard_cast_bf16_kernel<<<cgrid, 256, 0, stream>>>(cast);
+        }
     } else {
         for (int r = 0; r < nrel; ++r) {
             lard::Fp32Params p;
@@ -500,6 +562,19 @@ lard_status lard_kl_bwd_multi(const lard_relation* rel, int nrel, lard_dtype dty
     return kl_bwd(rel, nrel, dtype, B, n, d, tau, causal, grad_scale, stream);
 }
 
+size_t lard_kl_bwd_bf16_workspace_bytes(const lard_relation* rel, int nrel, int B, int n, int d) {
+    return bf16_workspace_bytes(rel, nrel, B, n, d);
+}
+
+lard_status lard_kl_bwd_multi_bf16(const lard_relation* rel, const lard_grads_bf16* out, int nrel,
+                                   lard_dtype dtype, int B, int n, int d, float tau, int causal,
+                                   float grad_scale, void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+    if (!out) return LARD_ERR_INVALID_ARG;
+    const Bf16Grads b16{out, workspace, workspace_bytes};
+    return kl_bwd(rel, nrel, dtype, B, n, d, tau, causal, grad_scale, stream, &b16);
+}
+
 const char* lard_status_string(lard_status s) {
     switch (s) {
         case LARD_OK: return "LARD_OK";
@@ -513,6 +588,12 @@ const char* lard_status_string(lard_status s) {
 
 lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return LARD_ERR_CUDA;
+    // The fault word to read is the one on the stream's GPU, which need not be
+    // the current device.
+    int dev = 0;
+    if (cudaStreamGetDevice(stream, &dev) != cudaSuccess) return LARD_ERR_CUDA;
+    DeviceGuard guard;
+    if (cudaSetDevice(dev) != cudaSuccess) return LARD_ERR_CUDA;
     unsigned int v = 0;
     if (cudaMemcpyFromSymbol(&v, lard::g_lard_fault, sizeof(v)) != cudaSuccess) return LARD_ERR_CUDA;
     if (fault_bits) *fault_bits = v;

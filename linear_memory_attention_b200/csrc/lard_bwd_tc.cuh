@@ -13,7 +13,9 @@
 // shared memory and added to HBM with TMA bulk reduce-adds (fp32 adds in L2,
 // whole 128-byte lines, rows past n clipped by the tensor map).  For a fused
 // self-relation the finished dY_s[J] is added into the same buffer the same
-// way; otherwise it is stored to dY_s.
+// way; otherwise it is stored to dY_s, in fp32 or rounded once to bf16.  With
+// bf16 gradient outputs the dX_s reduce-adds go to a caller-provided fp32
+// workspace, which lard_cast_bf16_kernel rounds to bf16 after this kernel.
 // The kernel is bound by shared-memory bandwidth: per tile the four SS GEMMs
 // read 256 KB of operands, and TMA writes, dZ stores and the dX staging add
 // another 224 KB; the GEMMs share the SM's shared-memory bandwidth with them.
@@ -40,20 +42,22 @@ namespace lard {
 struct TcBwdRel {
     const float* lse_t;
     const float* lse_s;
-    float* dYs;
-    int fuse_dy;  // 1: add dY_s into the dX_s buffer (self-relation total gradient), dYs unused
+    float* dYs;               // fp32 dY_s output, or
+    __nv_bfloat16* dYs_bf16;  // bf16 dY_s output (rounded once from the TMEM accumulator)
+    int fuse_dy;  // 1: add dY_s into the dX_s accumulator (self-relation total gradient), no dY_s output
     int block0;   // first grid block of this relation (its B*H*T blocks follow)
 };
 
 // A launch: up to kMaxRelations relations of equal n and d in one grid.
 struct TcBwdGroup {
     CUtensorMap xt[kMaxRelations], yt[kMaxRelations], xs[kMaxRelations], ys[kMaxRelations];
-    CUtensorMap dx[kMaxRelations];  // fp32 dX_s, for the reduce-adds
+    CUtensorMap dx[kMaxRelations];  // fp32 dX_s accumulator (the output, or a workspace), for the reduce-adds
     TcBwdRel rel[kMaxRelations];
     int nrel, n, T, causal;
     float cfac;      // tau * log2(e)
     float dz_scale;  // tau * grad_scale / n: dZ and the chain-rule tau in one factor
-    unsigned long long wait_ns;
+    unsigned long long wait_ns;   // limit of each wait inside the loops
+    unsigned long long drain_ns;  // limit of each drain on the way out (longer)
 };
 
 template <int D>
@@ -118,10 +122,11 @@ __global__ void __launch_bounds__(512, 1)
         float cfac, dz_scale;
         const float *lse_t, *lse_s;
         float* dYs;
+        __nv_bfloat16* dYs_bf16;
         int fuse_dy;
-        unsigned long long wait_ns;
+        unsigned long long wait_ns, drain_ns;
     } p = {g.n, g.T, g.causal, g.cfac, g.dz_scale, g.rel[rel].lse_t, g.rel[rel].lse_s, g.rel[rel].dYs,
-           g.rel[rel].fuse_dy, g.wait_ns};
+           g.rel[rel].dYs_bf16, g.rel[rel].fuse_dy, g.wait_ns, g.drain_ns};
     const int local = static_cast<int>(blockIdx.x) - g.rel[rel].block0;
     const int bh = local / p.T;
     const int J = local % p.T;
@@ -162,7 +167,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    const uint64_t lim = p.wait_ns;
+    const uint64_t lim = p.wait_ns, dlim = p.drain_ns;
     if (warp < 4) {
       ptx::regs_dec<kBwdRegsCtl>();
       if (warp == 0) {
@@ -204,11 +209,11 @@ __global__ void __launch_bounds__(512, 1)
             ++issued_s;
         }
         // Let every copy this warp started land before the block can exit.
-        ptx::mbar_drain(&ctrl->y_full, 0, lim);
-        if (issued_t > 0) ptx::mbar_drain(&ctrl->xt_full, (issued_t - 1) & 1, lim);
+        drain(&ctrl->y_full, 0, dlim);
+        if (issued_t > 0) drain(&ctrl->xt_full, (issued_t - 1) & 1, dlim);
         for (int s = 0; s < 2 && s < issued_s; ++s) {
             const int last = s + 2 * ((issued_s - 1 - s) / 2);
-            ptx::mbar_drain(&ctrl->xs_full[s], (last >> 1) & 1, lim);
+            drain(&ctrl->xs_full[s], (last >> 1) & 1, dlim);
         }
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(512, 1)
             ptx::umma_commit(&ctrl->mma_done);
         }
         __syncwarp();
-        ptx::mbar_drain(&ctrl->mma_done, 0, lim);
+        drain(&ctrl->mma_done, 0, dlim);
       }
     } else if (warp < 12) {
         ptx::regs_inc<kBwdRegsDz>();
@@ -449,7 +454,7 @@ __global__ void __launch_bounds__(512, 1)
             ptx::tc_fence_after();
             const int j = J * 128 + r;
             const int y0 = J * 128 + q * 32;
-            float* dst = p.fuse_dy ? nullptr : p.dYs + (static_cast<size_t>(bh) * p.n + (j < p.n ? j : 0)) * D;
+            const size_t row = (static_cast<size_t>(bh) * p.n + (j < p.n ? j : 0)) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float v[32];
@@ -459,10 +464,21 @@ __global__ void __launch_bounds__(512, 1)
                 if (p.fuse_dy) {
                     if (y0 < p.n) reduce_box(v, c, y0);
                 } else if (j < p.n) {
+                    if (p.dYs_bf16) {  // dY_s[J] is complete here: round it once
+                        uint4* dst = reinterpret_cast<uint4*>(p.dYs_bf16 + row + c * 32);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        *reinterpret_cast<float4*>(dst + c * 32 + 4 * u) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        for (int u = 0; u < 4; ++u)
+                            dst[u] = make_uint4(ptx::pack_bf16x2(v[8 * u], v[8 * u + 1]),
+                                                ptx::pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                                ptx::pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                                                ptx::pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+                    } else {
+                        float* dst = p.dYs + row + c * 32;
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4*>(dst + 4 * u) =
+                                make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    }
                 }
             }
         }

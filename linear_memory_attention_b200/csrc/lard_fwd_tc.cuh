@@ -59,7 +59,8 @@ struct TcFwdGroup {
     int nrel, n, T, causal;
     float cfac;  // tau * log2(e): S -> log2-domain logit
     float tau;
-    unsigned long long wait_ns;
+    unsigned long long wait_ns;   // limit of each wait inside the loops
+    unsigned long long drain_ns;  // limit of each drain on the way out (longer)
 };
 
 template <int D>
@@ -121,9 +122,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float cfac, tau;
         const __nv_bfloat16 *Xt, *Xs;
         float *lse_t, *lse_s, *row_kl;
-        unsigned long long wait_ns;
+        unsigned long long wait_ns, drain_ns;
     } p = {g.n, g.T, g.causal, g.cfac, g.tau, g.rel[rel].Xt, g.rel[rel].Xs, g.rel[rel].lse_t,
-           g.rel[rel].lse_s, g.rel[rel].row_kl, g.wait_ns};
+           g.rel[rel].lse_s, g.rel[rel].row_kl, g.wait_ns, g.drain_ns};
     const int local = static_cast<int>(blockIdx.x) - g.rel[rel].block0;
     const int bh = local / p.T;
     const int I = p.T - 1 - local % p.T;
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = ctrl->tmem_base;
-    const uint64_t lim = p.wait_ns;
+    const uint64_t lim = p.wait_ns, dlim = p.drain_ns;
 
     if (warp < 4) {
       ptx::regs_dec<kFwdRegsCtl>();
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // Let every copy this warp started land before the block can exit.
         for (int s = 0; s < L::NS && s < issued; ++s) {
             const int last = s + L::NS * ((issued - 1 - s) / L::NS);
-            ptx::mbar_drain(&ctrl->y_full[s], (last / L::NS) & 1, lim);
+            drain(&ctrl->y_full[s], (last / L::NS) & 1, dlim);
         }
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         if (lane == 0) ptx::umma_commit(&ctrl->mma_done);
         __syncwarp();
-        ptx::mbar_drain(&ctrl->mma_done, 0, lim);
+        drain(&ctrl->mma_done, 0, dlim);
       }
     } else {
         ptx::regs_inc<kFwdRegsStat>();

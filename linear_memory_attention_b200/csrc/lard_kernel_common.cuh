@@ -17,7 +17,16 @@ constexpr unsigned int kFaultBwdProducer = 1u << 4;
 constexpr unsigned int kFaultBwdMma = 1u << 5;
 constexpr unsigned int kFaultBwdSoftmax = 1u << 6;
 constexpr unsigned int kFaultBwdEpilogue = 1u << 7;
+constexpr unsigned int kFaultDrain = 1u << 8;  // a block exited before its own copies or MMAs finished
 constexpr unsigned int kFaultSelfTest = 1u << 15;
+
+// Wait on the way out for copies and MMAs this block started (ptx::mbar_drain,
+// which ignores the abort flag).  A drain that runs out of time means the
+// block may leave while the hardware still writes its shared memory or TMEM,
+// so it is reported on its own bit.
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (!ptx::mbar_drain(bar, parity, limit_ns)) atomicOr(&g_lard_fault, kFaultDrain);
+}
 
 // Relations (X/Y pairs of equal n and d, any head counts) that one launch of a
 // tensor-core kernel may cover; their blocks are laid out one relation after

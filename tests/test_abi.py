@@ -8,11 +8,12 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "lard.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "lard_probe.h")
 
 
-def declared_entry_points():
-    text = open(HEADER).read()
-    return re.findall(r"LARD_API\s+[\w\s\*]+?\b(lard_\w+)\s*\(", text)
+def declared_entry_points(header=HEADER, api="LARD_API"):
+    text = open(header).read()
+    return re.findall(api + r"\s+[\w\s\*]+?\b(lard_\w+)\s*\(", text)
 
 
 @pytest.fixture(scope="module")
@@ -38,6 +39,21 @@ def test_library_exports_every_declared_symbol(lib):
 def test_binding_lists_every_export():
     from linear_memory_attention_b200 import lard
     assert set(declared_entry_points()) == set(lard.EXPORTS)
+
+
+def test_probe_library_exports_its_header():
+    """The exponential-unit probe library (used by the benchmark) exports what
+    include/lard_probe.h declares; no compute call without a GPU."""
+    from linear_memory_attention_b200 import build, probe
+    build.build()
+    names = declared_entry_points(PROBE_HEADER, "LARD_PROBE_API")
+    assert names and set(names) == set(probe.EXPORTS)
+    for name in names:
+        assert hasattr(probe._lib, name)
+    # argument errors return before any CUDA call
+    ms, ex = ctypes.c_float(), ctypes.c_double()
+    assert probe._lib.lard_probe_exp_rate(5, 1, 1, ctypes.byref(ms), ctypes.byref(ex), None) == 1
+    assert probe._lib.lard_probe_exp_rate(0, 0, 1, ctypes.byref(ms), ctypes.byref(ex), None) == 1
 
 
 def test_status_strings_and_version(lib):
@@ -178,18 +194,110 @@ def test_binding_marshalling_errors():
     b = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16)
     f = torch.zeros((1, 2, 64, 128), dtype=torch.float16)
     with pytest.raises(ValueError):
-        lard._relations([])                                   # no relation
+        lard._relations([], "fwd")                                   # no relation
     with pytest.raises(ValueError):
-        lard._relations([dict(Xt=a, Xs=a)] * 5)               # more than LARD_MAX_RELATIONS
+        lard._relations([dict(Xt=a, Xs=a)] * 5, "fwd")               # more than LARD_MAX_RELATIONS
     with pytest.raises(ValueError):
-        lard._relations([dict(Xt=a, Xs=a), dict(Xt=b, Xs=b)])  # relations of different d
+        lard._relations([dict(Xt=a, Xs=a), dict(Xt=b, Xs=b)], "fwd")  # relations of different d
     with pytest.raises(ValueError):
-        lard._relations([dict(Xt=a, Xs=b)])                   # X_t and X_s of different shapes
+        lard._relations([dict(Xt=a, Xs=b)], "fwd")                   # X_t and X_s of different shapes
     with pytest.raises(ValueError):
-        lard._shape(f)                                        # unsupported dtype
+        lard._shape(f)                                               # unsupported dtype
     with pytest.raises(ValueError):
-        lard._shape(a[0])                                     # not [B, H, n, d]
-    arr, dt, B, n, d = lard._relations([dict(Xt=a, Xs=a), dict(Xt=a[:, :1].contiguous(),
-                                                                Xs=a[:, :1].contiguous())])
+        lard._shape(a[0])                                            # not [B, H, n, d]
+    a1 = a[:, :1].contiguous()
+    outs = lambda H: dict(lse_t=torch.empty(1, H, 64), lse_s=torch.empty(1, H, 64),  # noqa: E731
+                          row_kl=torch.empty(1, H, 64), loss_bh=torch.empty(H),
+                          dXs=torch.empty(1, H, 64, 128), dYs=torch.empty(1, H, 64, 128))
+    arr, dt, B, n, d = lard._relations([dict(Xt=a, Xs=a, **outs(2)), dict(Xt=a1, Xs=a1, **outs(1))],
+                                       "fwd")
     assert (dt, B, n, d) == (lard.LARD_DTYPE_BF16, 1, 64, 128)
-    assert arr[0].H == 2 and arr[1].H == 1 and arr[0].Yt == arr[0].Xt and arr[1].dYs is None
+    assert arr[0].H == 2 and arr[1].H == 1 and arr[0].Yt == arr[0].Xt
+    assert arr[1].dXs is None and arr[1].dYs is None                 # a phase passes only its outputs
+    arr, *_ = lard._relations([dict(Xt=a, Xs=a, **dict(outs(2), dYs=None))], "bwd")
+    assert arr[0].dYs is None and arr[0].row_kl is None and arr[0].dXs is not None
+
+
+@pytest.mark.parametrize("field,bad", [
+    ("dXs", lambda: torch_zeros((1, 2, 64, 128), "bfloat16")),     # wrong dtype
+    ("dXs", lambda: torch_zeros((1, 2, 64, 64), "float32")),       # short
+    ("dYs", lambda: torch_zeros((1, 2, 128, 64), "float32")[:, :, ::2]),  # right size, not contiguous
+    ("lse_t", lambda: torch_zeros((1, 2, 63), "float32")),         # short
+    ("lse_s", lambda: torch_zeros((1, 2, 64), "float64")),         # wrong dtype
+    ("row_kl", lambda: None),                                      # missing
+    ("loss_bh", lambda: torch_zeros((3,), "float32")),             # wrong length
+])
+def test_binding_checks_every_output(field, bad):
+    """Every output buffer is checked for dtype, size, contiguity and device: the
+    library cannot see buffer sizes, so a short or wrong-typed buffer would be
+    written past its end."""
+    import torch
+    from linear_memory_attention_b200 import lard
+    a = torch.zeros((1, 2, 64, 128), dtype=torch.bfloat16)
+    good = dict(lse_t=torch.empty(1, 2, 64), lse_s=torch.empty(1, 2, 64), row_kl=torch.empty(1, 2, 64),
+                loss_bh=torch.empty(2), dXs=torch.empty(1, 2, 64, 128), dYs=torch.empty(1, 2, 64, 128))
+    rel = dict(Xt=a, Xs=a, **dict(good, **{field: bad()}))
+    phase = "bwd" if field in ("dXs", "dYs") else "fwd"
+    with pytest.raises(ValueError):
+        lard._relations([rel], phase)
+    if field in ("dXs",):
+        with pytest.raises(ValueError):
+            lard.lard_kl_bwd(a, a, a, a, 0.1, True, good["lse_t"], good["lse_s"], 1.0, rel["dXs"],
+                             good["dYs"])
+        with pytest.raises(ValueError):
+            lard.lard_kl_bwd_self(a, a, 0.1, True, good["lse_t"], good["lse_s"], 1.0, rel["dXs"])
+    if field in ("lse_t", "row_kl", "loss_bh"):
+        kw = dict(good)
+        kw[field] = rel[field]
+        with pytest.raises(ValueError):
+            lard.lard_kl_fwd(a, a, a, a, 0.1, True, kw["lse_t"], kw["lse_s"], kw["row_kl"], kw["loss_bh"])
+    with pytest.raises(ValueError):
+        lard.lard_kl_fwd_multi([dict(Xt=a, Xs=a, **good)], 0.1, True, loss_total=torch.empty(2))
+
+
+def torch_zeros(shape, dtype):
+    import torch
+    return torch.zeros(shape, dtype=getattr(torch, dtype))
+
+
+def bwd_multi_bf16(lib, specs, outs, ws=0x1d000000, ws_bytes=None, dtype=0, n=300, d=128, g=1.0):
+    from linear_memory_attention_b200.lard import _Bf16Grads
+    arr = relations(specs)
+    o = (_Bf16Grads * max(1, len(outs)))()
+    for k, (x, y) in enumerate(outs):
+        o[k].dXs, o[k].dYs = x, y
+    if ws_bytes is None:
+        ws_bytes = lib.lard_kl_bwd_bf16_workspace_bytes(arr, len(specs), 1, n, d)
+    return lib.lard_kl_bwd_multi_bf16(arr, o, len(specs), dtype, 1, n, d, ctypes.c_float(0.088), 1,
+                                      ctypes.c_float(g), ws, ws_bytes, None)
+
+
+BF0 = dict(REL0, dXs=None, dYs=None)
+BF1 = dict(REL1, dXs=None, dYs=None)
+OUT0, OUT1 = (0x20000000, 0x21000000), (0x22000000, None)
+
+
+def test_bf16_workspace_bytes(lib):
+    assert lib.lard_kl_bwd_bf16_workspace_bytes(relations([BF0, BF1]), 2, 1, 300, 128) == (2 + 1) * 300 * 128 * 4
+    assert lib.lard_kl_bwd_bf16_workspace_bytes(relations([BF0]), 1, 3, 300, 64) == 3 * 2 * 300 * 64 * 4
+    assert lib.lard_kl_bwd_bf16_workspace_bytes(relations([BF0]), 0, 1, 300, 128) == 0
+    assert lib.lard_kl_bwd_bf16_workspace_bytes(relations([dict(BF0, H=0)]), 1, 1, 300, 128) == 0
+    assert lib.lard_kl_bwd_bf16_workspace_bytes(None, 1, 1, 300, 128) == 0
+
+
+@pytest.mark.parametrize("specs,outs,kw,code", [
+    ([BF0, BF1], [OUT0, OUT1], dict(dtype=1), 2),                     # fp32 inputs: full-precision path only
+    ([BF0, BF1], [OUT0, OUT1], dict(ws_bytes=100), 1),                # workspace too small
+    ([BF0, BF1], [OUT0, OUT1], dict(ws=0x1d000008), 1),               # misaligned workspace
+    ([BF0, BF1], [OUT0, OUT1], dict(ws=0), 1),                        # no workspace
+    ([BF0, BF1], [OUT0, OUT1], dict(ws=0x20000000), 1),               # workspace over an output
+    ([BF0, BF1], [OUT0, (0x20000000 + 4096, None)], {}, 1),           # two outputs overlap
+    ([BF0, BF1], [(None, 0x21000000), OUT1], {}, 1),                  # dXs missing
+    ([dict(BF0, dXs=O5), BF1], [OUT0, OUT1], {}, 1),                  # fp32 field set as well
+    ([BF0, BF1], [(0x20000008, 0x21000000), OUT1], {}, 1),            # misaligned bf16 output
+    ([BF0, dict(BF1, Ys=0x700000)], [OUT0, OUT1], {}, 1),             # fused needs Y = X
+    ([BF0, BF1], [OUT0, OUT1], dict(g=float("nan")), 1),
+    ([BF0, BF1], [OUT0, OUT1], dict(d=96), 2),
+])
+def test_bwd_multi_bf16_rejects_bad_arguments(lib, specs, outs, kw, code):
+    assert bwd_multi_bf16(lib, specs, outs, **kw) == code

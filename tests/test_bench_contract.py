@@ -37,12 +37,14 @@ def test_reference_arm_line():
 
 
 @pytest.mark.gpu
-def test_product_arm_line():
+@pytest.mark.parametrize("grads", ["partials", "dq"])
+def test_product_arm_line(grads):
     import torch
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     K = 4
-    d = _run(["--workload", "n4096", "--steps", str(K), "--warmup", "3", "--cpu-seconds", "1"], 900)
+    d = _run(["--workload", "n4096", "--steps", str(K), "--warmup", "3", "--cpu-seconds", "1",
+              "--grads", grads], 900)
     for k in COMMON + ("roofline", "clocks", "gpu_launches", "extra_hbm", "tflops", "kernel_ms"):
         assert k in d, k
     assert d["n_gpus"] == 1 and d["steps"] == K and d["warmup"] == 3 and d["scaling"] == "weak"
@@ -52,12 +54,30 @@ def test_product_arm_line():
         assert k in r, k
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert 0 < r["frac"] < 1.5 and math.isclose(r["frac"], r["achieved"] / r["peak"], rel_tol=1e-9)
+    assert r["cycles_per_tile"] > r["tensor_cycles_per_tile"] > 0
+    p1 = d["phase1_roofline"]
+    assert p1["bound"] == "alu" and p1["measured_ex2_per_clk_per_sm"] > 0 and 0 < p1["frac"] < 1.5
     e = d["e2e"]
-    assert e["value"] > 0 and e["unit"] == d["unit"] and e["d2h_bytes_per_step"] == 4
+    grads_bytes = (1 if grads == "dq" else 2) * 3 * 32 * 4096 * 128 * 4
+    assert e["value"] > 0 and e["unit"] == d["unit"] and e["d2h_bytes_per_step"] == grads_bytes + 4
     assert e["h2d_bytes_per_step"] == 6 * 32 * 4096 * 128 * 2  # six bf16 input tensors per step
     assert d["gpu_launches"] == 4 * K
-    assert d["extra_hbm"]["state_bytes"] == 12 * 3 * 32 * 4096
-    assert d["extra_hbm"]["allocated_per_step_bytes"] == 0
+    x = d["extra_hbm"]
+    assert x["state_bytes"] == x["state_bytes_expected"] == 12 * 3 * 32 * 4096 + 4 * 3 * 32
+    assert x["allocated_per_step_bytes"] == 0 and x["torch_peak_above_buffers_bytes"] == 0
     assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0 and cb["unit"] == d["unit"]
+
+
+@pytest.mark.gpu
+def test_product_arm_job_split_one_rank():
+    """--scaling strong on one GPU: the one rank's slice is the whole job."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    d = _run(["--workload", "gqa-n8000", "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+              "--scaling", "strong", "--no-probe"], 900)
+    assert d["scaling"] == "strong" and d["n_gpus"] == 1 and d["value"] > 0
+    assert d["config"]["parallelism"].startswith("units1")
+    assert d["extra_hbm"]["rows"] == 2 * (32 + 8 + 8) * 8000

@@ -1,13 +1,17 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
 Small cases compare every output element by element; they span several
-128 x 128 tiles, ragged tails, n = 1 and both masks.  The five workloads are
-run at their full sizes in the launch configuration the benchmark uses; the
-oracle then checks sampled heads or sampled rows (tail rows give the exact
-dY_s of the tail columns), and properties that hold at any size are checked
-on every output.
+128 x 128 tiles, ragged tails, n = 1 and both masks.  The five workloads run
+at their full sizes through the grouped call the benchmark times (one
+lard_kl_fwd_multi and one lard_kl_bwd_multi launch over all relations); the
+oracle, run over row chunks, checks sampled heads whole (every row, and dY_s
+on every column), the fused self-relation gradient of one head, and
+properties that hold at any size are checked on every output.  The single-
+relation calls are checked at n = 4096, and a 131072-long head on sampled and
+tail rows.
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -15,7 +19,7 @@ import torch
 
 import oracle
 from parity_util import (TOL, assert_close_abs, assert_grad_close, assert_kl_close, assert_rel,
-                         compare_full, f64, gpu_relation, grad_floor, random_cross)
+                         compare_full, f64, gpu_relation, grad_floor, oracle_head, random_cross)
 from linear_memory_attention_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -125,8 +129,9 @@ def test_extra_memory_is_linear(lard):
 # ------------------------------------------------------------------ workloads at full size
 
 def _run_workload(lard, w, check):
-    """Run every relation of a workload through the C ABI (one at a time, so
-    that host and device memory stay bounded) and hand each to ``check``."""
+    """Run every relation of a workload through the single-relation C ABI calls
+    (one at a time, so that host and device memory stay bounded) and hand
+    each to ``check``."""
     for rel in w.relations:
         Xt, Xs = synth.make_relation(w, rel)
         xt, xs = Xt.cuda(), Xs.cuda()
@@ -134,6 +139,7 @@ def _run_workload(lard, w, check):
         torch.cuda.synchronize()
         lard.lard_device_status()
         _properties(xs, g, w, f"{w.name} {rel}")
+        assert_rel(g["loss"].item(), g["loss_bh"].double().sum().item(), 1e-5, f"{w.name} {rel} loss total")
         check(rel, Xt, Xs, g)
         del g, xt, xs
         torch.cuda.empty_cache()
@@ -146,7 +152,6 @@ def _properties(xs, g, w, what):
     kl = g["row_kl"].double()
     assert kl.min().item() >= -1e-4, f"{what}: KL must be non-negative"
     torch.testing.assert_close(g["loss_bh"].double(), kl.reshape(-1, w.n).mean(-1), rtol=1e-5, atol=1e-9)
-    assert_rel(g["loss"].item(), g["loss_bh"].double().sum().item(), 1e-5, what + " loss total")
     x = xs.double()
     zdiag = w.tau * (x * x).sum(-1)
     assert bool((g["lse_s"].double() >= zdiag - 1e-3).all()), f"{what}: LSE_s below the diagonal logit"
@@ -161,22 +166,103 @@ def _host(t):
     return t.detach().to("cpu").to(torch.float64).numpy()
 
 
-def _check_heads(w, heads):
+def _compare_head(got, o, w, what, floor):
+    """Element-by-element comparison of one whole head (all rows, all columns)."""
     tol = TOL[w.dtype]
+    assert_close_abs(got["lse_t"], o["lse_t"], tol["lse"], what + " lse_t")
+    assert_close_abs(got["lse_s"], o["lse_s"], tol["lse"], what + " lse_s")
+    assert_kl_close(got["row_kl"], o["row_kl"], tol, what + " row_kl")
+    assert_rel(got["loss_bh"], o["loss"], tol["loss"], what + " loss", tol["loss_abs"])
+    assert_grad_close(got["dXs"], o["dXs"], tol["grad"], what + " dXs", floor)
+    assert_grad_close(got["dYs"], o["dYs"], tol["grad"], what + " dYs (every column)", floor)
 
+
+def _grouped_workload(lard, w, heads, fused_head=None, bf16=False):
+    """The launch the benchmark times: every relation of the workload in one
+    lard_kl_fwd_multi and one lard_kl_bwd_multi call.  Properties that hold at
+    any size are checked on every output; the sampled heads (``heads``: relation
+    -> [(b, h)]) are compared whole, every row and every column of dY_s, with
+    the oracle run over row chunks.  ``fused_head`` = (relation, b, h) also runs
+    the grouped call with the fused self-relation gradient and compares that
+    head's dQ = dX_s + dY_s with the oracle's sum.  ``bf16`` repeats both
+    grouped calls with bf16 gradient outputs (lard_kl_bwd_multi_bf16) and
+    compares the same heads."""
+    host = synth.make_all(w)
+    pairs = [(host[r][0].cuda(), host[r][1].cuda()) for r in w.relations]
+    outs, loss = lard.relations_kl(pairs, w.tau, w.causal)
+    torch.cuda.synchronize()
+    lard.lard_device_status()
+    total = 0.0
+    got = {}
+    for rel, (xt, xs), g in zip(w.relations, pairs, outs):
+        _properties(xs, g, w, f"{w.name} {rel}")
+        total += g["loss_bh"].double().sum().item()
+        H = xt.shape[1]
+        for (b, h) in heads.get(rel, []):
+            got[(rel, b, h)] = {"lse_t": _host(g["lse_t"][b, h]), "lse_s": _host(g["lse_s"][b, h]),
+                                "row_kl": _host(g["row_kl"][b, h]),
+                                "loss_bh": g["loss_bh"][b * H + h].item(),
+                                "dXs": _host(g["dXs"][b, h]), "dYs": _host(g["dYs"][b, h])}
+    assert_rel(loss.item(), total, 1e-5, f"{w.name} summed loss of the grouped call")
+    del outs
+    torch.cuda.empty_cache()
+    dq, got16, dq16 = None, {}, None
+    if fused_head is not None:
+        outs_f, loss_f = lard.relations_kl(pairs, w.tau, w.causal, fused_self=True)
+        torch.cuda.synchronize()
+        lard.lard_device_status()
+        assert loss_f.item() == loss.item(), "Phase 1 of the fused call must repeat the loss bit for bit"
+        rel, b, h = fused_head
+        dq = _host(outs_f[w.relations.index(rel)]["dXs"][b, h])
+        del outs_f
+        torch.cuda.empty_cache()
+    if bf16:
+        outs16, _ = lard.relations_kl(pairs, w.tau, w.causal, grad_dtype="bf16")
+        torch.cuda.synchronize()
+        lard.lard_device_status()
+        for rel, g in zip(w.relations, outs16):
+            assert g["dXs"].dtype == torch.bfloat16 and g["dYs"].dtype == torch.bfloat16
+            for (b, h) in heads.get(rel, []):
+                got16[(rel, b, h)] = (_host(g["dXs"][b, h]), _host(g["dYs"][b, h]))
+        del outs16
+        torch.cuda.empty_cache()
+        if fused_head is not None:
+            outs16, _ = lard.relations_kl(pairs, w.tau, w.causal, fused_self=True, grad_dtype="bf16")
+            torch.cuda.synchronize()
+            lard.lard_device_status()
+            rel, b, h = fused_head
+            dq16 = _host(outs16[w.relations.index(rel)]["dXs"][b, h])
+            del outs16
+    del pairs
+    torch.cuda.empty_cache()
+    for (rel, b, h), g in got.items():
+        xt, xs = f64(host[rel][0][b, h]), f64(host[rel][1][b, h])
+        o = oracle_head(xt, xs, w.tau, w.causal)
+        what = f"{w.name} {rel} head ({b},{h}) grouped launch"
+        floor = grad_floor(xs, xs, w.tau, 1.0, w.n)
+        _compare_head(g, o, w, what, floor)
+        if fused_head == (rel, b, h):
+            assert_grad_close(dq, o["dXs"] + o["dYs"], TOL[w.dtype]["grad"], what + " fused dQ", floor)
+            if dq16 is not None:
+                assert_grad_close(dq16, o["dXs"] + o["dYs"], TOL[w.dtype]["grad"], what + " fused dQ (bf16)",
+                                  floor)
+        if (rel, b, h) in got16:
+            gx, gy = got16[(rel, b, h)]
+            assert_grad_close(gx, o["dXs"], TOL[w.dtype]["grad"], what + " dXs (bf16)", floor)
+            assert_grad_close(gy, o["dYs"], TOL[w.dtype]["grad"], what + " dYs (bf16, every column)", floor)
+
+
+def _check_heads(w, heads):
+    """Whole heads of a single-relation call against the oracle."""
     def check(rel, Xt, Xs, g):
         H = Xt.shape[1]
         for (b, h) in heads[rel]:
             xt, xs = f64(Xt[b, h]), f64(Xs[b, h])
             o = oracle.relation(xt, xt, xs, xs, w.tau, w.causal)
-            what = f"{w.name} {rel} head ({b},{h})"
-            assert_close_abs(_host(g["lse_t"][b, h]), o["lse_t"], tol["lse"], what + " lse_t")
-            assert_close_abs(_host(g["lse_s"][b, h]), o["lse_s"], tol["lse"], what + " lse_s")
-            assert_kl_close(_host(g["row_kl"][b, h]), o["row_kl"], tol, what + " row_kl")
-            assert_rel(g["loss_bh"][b * H + h].item(), o["loss"], tol["loss"], what + " loss", tol["loss_abs"])
-            floor = grad_floor(xs, xs, w.tau, 1.0, w.n)
-            assert_grad_close(_host(g["dXs"][b, h]), o["dXs"], tol["grad"], what + " dXs", floor)
-            assert_grad_close(_host(g["dYs"][b, h]), o["dYs"], tol["grad"], what + " dYs", floor)
+            got = {"lse_t": _host(g["lse_t"][b, h]), "lse_s": _host(g["lse_s"][b, h]),
+                   "row_kl": _host(g["row_kl"][b, h]), "loss_bh": g["loss_bh"][b * H + h].item(),
+                   "dXs": _host(g["dXs"][b, h]), "dYs": _host(g["dYs"][b, h])}
+            _compare_head(got, o, w, f"{w.name} {rel} head ({b},{h})", grad_floor(xs, xs, w.tau, 1.0, w.n))
     return check
 
 
@@ -212,6 +298,8 @@ def _check_rows(w, heads, n_tail, n_random, seed):
 
 
 def test_workload_fp32_small(lard):
+    """The fp32 workload (one relation): whole relation, every head, through the
+    single-relation calls and through the grouped call."""
     w = synth.WORKLOADS["fp32-small"]
 
     def check(rel, Xt, Xs, g):
@@ -219,29 +307,61 @@ def test_workload_fp32_small(lard):
         compare_full({k: _host(v) for k, v in g.items()}, o, "fp32", f"{w.name} {rel}",
                      grad_floor(f64(Xs), f64(Xs), w.tau, 1.0, w.n))
     _run_workload(lard, w, check)
+    _grouped_workload(lard, w, {"Q": [(0, 0), (0, 1)]})
 
 
 def test_workload_n4096(lard):
+    """B1 H32 n4096 d128, three relations, grouped launch: two whole heads per
+    relation, and one head's fused dQ."""
     w = synth.WORKLOADS["n4096"]
-    _run_workload(lard, w, _check_heads(w, {r: [(0, 0), (0, 31)] for r in w.relations}))
+    _grouped_workload(lard, w, {r: [(0, 0), (0, 31)] for r in w.relations}, fused_head=("K", 0, 31),
+                      bf16=True)
+
+
+def test_workload_n4096_single_relation_calls(lard):
+    """The same workload through one lard_kl_fwd / lard_kl_bwd call per relation."""
+    w = synth.WORKLOADS["n4096"]
+    _run_workload(lard, w, _check_heads(w, {r: [(0, 7)] for r in w.relations}))
 
 
 def test_workload_gqa_n8000(lard):
+    """GQA: B = 2, n = 8000 (62 full row blocks and a 64-row tail), 32 Q heads and
+    8 K/V heads in one grouped launch; five whole heads, one fused dQ."""
     w = synth.WORKLOADS["gqa-n8000"]
     heads = {"Q": [(0, 3), (1, 30)], "K": [(0, 0), (1, 7)], "V": [(1, 2)]}
-    _run_workload(lard, w, _check_rows(w, heads, n_tail=200, n_random=24, seed=5))
+    _grouped_workload(lard, w, heads, fused_head=("V", 1, 2), bf16=True)
+
+
+# The oracle checks a whole head at n = 32768 in about two minutes on 16 host
+# cores (n^2 explicit logits per map), at n = 16384 in about half a minute.
+# By default one whole head per relation is checked at each size, which keeps
+# the GPU test run well inside its time limit; LARD_PARITY_HEADS=full checks
+# two heads per relation at n = 32768 and four at n = 16384 (about 18 minutes
+# of oracle time).
+FULL_HEADS = os.environ.get("LARD_PARITY_HEADS") == "full"
 
 
 def test_workload_n16384(lard):
+    """B1 H32 n16384: whole heads (every row, every dY column), grouped launch."""
     w = synth.WORKLOADS["n16384"]
-    _run_workload(lard, w, _check_rows(w, {r: [(0, 5)] for r in w.relations}, n_tail=160,
-                                       n_random=16, seed=6))
+    if FULL_HEADS:
+        heads = {r: [(0, 0), (0, 5), (0, 18), (0, 31)] for r in w.relations}
+    else:
+        heads = {"Q": [(0, 5)], "K": [(0, 18)], "V": [(0, 31)]}
+    _grouped_workload(lard, w, heads)
 
 
 def test_workload_n32768(lard):
+    """The benchmark's workload, B1 H32 n32768, in the benchmark's launch
+    configuration: whole heads (every row; dY_s on every column, including the
+    early columns that accumulate over all 256 row blocks), the fused dQ of
+    one head, and the same with bf16 gradient outputs."""
     w = synth.WORKLOADS["n32768"]
-    _run_workload(lard, w, _check_rows(w, {r: [(0, 0), (0, 17)] for r in w.relations}, n_tail=160,
-                                       n_random=16, seed=7))
+    if FULL_HEADS:
+        heads = {r: [(0, 0), (0, 17)] for r in w.relations}
+    else:
+        heads = {"Q": [(0, 0)], "K": [(0, 17)], "V": [(0, 31)]}
+    _grouped_workload(lard, w, heads, fused_head=("Q", 0, 0), bf16=True)
 
 
 def test_long_single_head(lard):
