@@ -63,7 +63,9 @@ def test_product_arm_line(grads):
     assert e["h2d_bytes_per_step"] == 6 * 32 * 4096 * 128 * 2  # six bf16 input tensors per step
     assert d["gpu_launches"] == 4 * K
     x = d["extra_hbm"]
-    assert x["state_bytes"] == x["state_bytes_expected"] == 12 * 3 * 32 * 4096 + 4 * 3 * 32
+    assert x["state_bytes_expected"] == 12 * 3 * 32 * 4096 + 4 * 3 * 32
+    # the allocator rounds each of the 4 state buffers of a relation up to its 512-byte granule
+    assert x["state_bytes_expected"] <= x["state_bytes"] <= x["state_bytes_expected"] + 3 * 4 * 512
     assert x["allocated_per_step_bytes"] == 0 and x["torch_peak_above_buffers_bytes"] == 0
     assert set(d["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
     cb = d["cpu_baseline"]
