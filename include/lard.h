@@ -69,7 +69,9 @@ typedef enum {
     LARD_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, non-finite scalar, aliasing */
     LARD_ERR_UNSUPPORTED = 2, /* head dim or dtype not built, or a GPU other than sm_100 */
     LARD_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
-    LARD_ERR_TIMEOUT = 4      /* a kernel wait ran out of time (see lard_device_status) */
+    LARD_ERR_TIMEOUT = 4,     /* a kernel wait ran out of time (see lard_device_status) */
+    LARD_ERR_TOO_LARGE = 5    /* the problem needs more than the fixed workspace of
+                                 lard_kl_bwd_multi_bf16_noalloc */
 } lard_status;
 
 typedef enum { LARD_DTYPE_BF16 = 0, LARD_DTYPE_FP32 = 1 } lard_dtype;
@@ -235,6 +237,38 @@ LARD_API lard_status lard_kl_bwd_multi_bf16(const lard_relation* rel, const lard
                                    lard_dtype dtype, int B, int n, int d, float tau, int causal,
                                    float grad_scale, void* workspace, size_t workspace_bytes,
                                    cudaStream_t stream);
+
+/*
+ * lard_kl_bwd_multi_bf16 for callers that cannot allocate device memory.
+ *
+ * Some callers cannot call cudaMalloc at the point where they run Phase 2:
+ * code inside another framework's training step whose memory pool owns the
+ * whole device, or a runtime that forbids device allocation once it has
+ * started.  Such a caller cannot provide the fp32 workspace that
+ * lard_kl_bwd_multi_bf16 asks for.  This entry point takes the same
+ * arguments without the workspace and uses instead a fixed array in the
+ * library's device memory of LARD_NOALLOC_WORKSPACE_BYTES (64 MiB): every
+ * GPU that loads the library holds that array until the process exits.
+ * The pages that define the method have no counterpart of this entry point.
+ *
+ *   rel, out, nrel, dtype, B, n, d, tau, causal, grad_scale, stream: as for
+ *              lard_kl_bwd_multi_bf16.
+ * Limit: lard_kl_bwd_bf16_workspace_bytes(rel, nrel, B, n, d) must not exceed
+ * LARD_NOALLOC_WORKSPACE_BYTES (for example B * H * n * d summed over the
+ * relations <= 16 Mi elements: 32 heads of n = 4096, d = 128); a larger
+ * problem returns LARD_ERR_TOO_LARGE before anything is enqueued.
+ * The call allocates nothing: it looks up the array's device address on the
+ * first call on each GPU (so that first call should come before any stream
+ * capture), clears the part it uses on `stream`, and accumulates there.
+ * Every call on a GPU shares the one array, which keeps the last call's
+ * contents: calls whose work can overlap on the GPU (on different streams
+ * without ordering between them, or from several host threads) race on it
+ * and give wrong gradients.  Order such calls, for example on one stream.
+ */
+#define LARD_NOALLOC_WORKSPACE_BYTES (64u << 20)
+LARD_API lard_status lard_kl_bwd_multi_bf16_noalloc(const lard_relation* rel, const lard_grads_bf16* out,
+                                           int nrel, lard_dtype dtype, int B, int n, int d, float tau,
+                                           int causal, float grad_scale, cudaStream_t stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 LARD_API const char* lard_status_string(lard_status s);

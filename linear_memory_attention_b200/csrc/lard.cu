@@ -29,8 +29,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Workspace of lard_kl_bwd_multi_bf16_noalloc, for callers that cannot
+// allocate device memory: a file-scope device array, present on every GPU
+// that loads the library, shared by every call of that entry point on that
+// GPU.  Host code reaches it only through the device address that
+// cudaGetSymbolAddress returns (g_static_ws_ptr, set once per device).
+constexpr size_t kStaticWorkspaceBytes = size_t(64) << 20;  // 64 MiB
+static_assert(kStaticWorkspaceBytes == LARD_NOALLOC_WORKSPACE_BYTES, "workspace size differs from the header");
+static __device__ __align__(256) unsigned char g_lard_static_ws[kStaticWorkspaceBytes];
+
 std::mutex g_mu;
 bool g_ready[kMaxDevices];
+void* g_static_ws_ptr[kMaxDevices];
 lard_status g_dev_status[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 
@@ -566,6 +576,37 @@ size_t lard_kl_bwd_bf16_workspace_bytes(const lard_relation* rel, int nrel, int 
     return bf16_workspace_bytes(rel, nrel, B, n, d);
 }
 
+lard_status lard_kl_bwd_multi_bf16_noalloc(const lard_relation* rel, const lard_grads_bf16* out, int nrel,
+                                           lard_dtype dtype, int B, int n, int d, float tau, int causal,
+                                           float grad_scale, cudaStream_t stream) {
+    if (!rel || !out || nrel < 1 || nrel > lard::kMaxRelations || !rel[0].Xt) return LARD_ERR_INVALID_ARG;
+    const size_t need = bf16_workspace_bytes(rel, nrel, B, n, d);
+    if (need == 0) return LARD_ERR_INVALID_ARG;
+    if (need > kStaticWorkspaceBytes) return LARD_ERR_TOO_LARGE;
+    // The device address of this GPU's copy of the array, looked up once per
+    // device with that device current.
+    DeviceGuard guard;
+    lard_status st = select_device(rel[0].Xt);
+    if (st != LARD_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LARD_ERR_CUDA;
+    void* ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_static_ws_ptr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_lard_static_ws) != cudaSuccess || !p) {
+                cudaGetLastError();
+                return LARD_ERR_CUDA;
+            }
+            g_static_ws_ptr[dev] = p;
+        }
+        ws = g_static_ws_ptr[dev];
+    }
+    const Bf16Grads b16{out, ws, kStaticWorkspaceBytes};
+    return kl_bwd(rel, nrel, dtype, B, n, d, tau, causal, grad_scale, stream, &b16);
+}
+
 lard_status lard_kl_bwd_multi_bf16(const lard_relation* rel, const lard_grads_bf16* out, int nrel,
                                    lard_dtype dtype, int B, int n, int d, float tau, int causal,
                                    float grad_scale, void* workspace, size_t workspace_bytes,
@@ -582,6 +623,7 @@ const char* lard_status_string(lard_status s) {
         case LARD_ERR_UNSUPPORTED: return "LARD_ERR_UNSUPPORTED";
         case LARD_ERR_CUDA: return "LARD_ERR_CUDA";
         case LARD_ERR_TIMEOUT: return "LARD_ERR_TIMEOUT";
+        case LARD_ERR_TOO_LARGE: return "LARD_ERR_TOO_LARGE";
     }
     return "LARD_ERR_UNKNOWN";
 }

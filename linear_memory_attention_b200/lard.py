@@ -29,11 +29,13 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblard.so")
 
-LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT = range(5)
+LARD_OK, LARD_ERR_INVALID_ARG, LARD_ERR_UNSUPPORTED, LARD_ERR_CUDA, LARD_ERR_TIMEOUT, LARD_ERR_TOO_LARGE = range(6)
+LARD_NOALLOC_WORKSPACE_BYTES = 64 << 20
 LARD_DTYPE_BF16, LARD_DTYPE_FP32 = 0, 1
 
 EXPORTS = ("lard_kl_fwd", "lard_kl_bwd", "lard_kl_bwd_self", "lard_kl_fwd_multi",
            "lard_kl_bwd_multi", "lard_kl_bwd_bf16_workspace_bytes", "lard_kl_bwd_multi_bf16",
+           "lard_kl_bwd_multi_bf16_noalloc",
            "lard_status_string", "lard_device_status", "lard_selftest_timeout", "lard_version")
 LARD_MAX_RELATIONS = 4
 
@@ -80,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.lard_kl_bwd_bf16_workspace_bytes.argtypes = [rp, i, i, i, i]
     lib.lard_kl_bwd_multi_bf16.restype = i
     lib.lard_kl_bwd_multi_bf16.argtypes = [rp, g16p, i, i, i, i, i, f, i, f, vp, ctypes.c_size_t, vp]
+    lib.lard_kl_bwd_multi_bf16_noalloc.restype = i
+    lib.lard_kl_bwd_multi_bf16_noalloc.argtypes = [rp, g16p, i, i, i, i, i, f, i, f, vp]
     lib.lard_status_string.restype = ctypes.c_char_p
     lib.lard_status_string.argtypes = [i]
     lib.lard_device_status.restype = i
@@ -325,6 +329,27 @@ def lard_kl_bwd_multi_bf16(relations, tau, causal, grad_scale, workspace, stream
                                      _stream(stream, Xt0))
     if st != LARD_OK:
         raise LardError(st, "lard_kl_bwd_multi_bf16")
+
+
+def lard_kl_bwd_multi_bf16_noalloc(relations, tau, causal, grad_scale, stream=None):
+    """lard_kl_bwd_multi_bf16 without a workspace argument, for callers that cannot
+    allocate device memory: the library's fixed LARD_NOALLOC_WORKSPACE_BYTES array
+    is used instead.  Calls that can overlap on the GPU race on that array."""
+    import torch
+    arr, dt, B, n, d = _relations([{k: v for k, v in r.items() if k not in ("dXs", "dYs")}
+                                   for r in relations], "bwd_outputs_elsewhere")
+    out = (_Bf16Grads * len(relations))()
+    for k, r in enumerate(relations):
+        H = int(r["Xt"].shape[1])
+        _check_grad(r.get("dXs"), r["Xt"], H, "dXs", dtype=torch.bfloat16)
+        _check_grad(r.get("dYs"), r["Xt"], H, "dYs", dtype=torch.bfloat16, optional=True)
+        out[k].dXs = r["dXs"].data_ptr()
+        out[k].dYs = None if r.get("dYs") is None else r["dYs"].data_ptr()
+    st = _lib.lard_kl_bwd_multi_bf16_noalloc(arr, out, len(relations), dt, B, n, d, float(tau),
+                                             int(bool(causal)), float(grad_scale),
+                                             _stream(stream, relations[0]["Xt"]))
+    if st != LARD_OK:
+        raise LardError(st, "lard_kl_bwd_multi_bf16_noalloc")
 
 
 def relations_kl(pairs, tau, causal=True, grad_scale=1.0, backward=True, fused_self=False,

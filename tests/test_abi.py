@@ -58,9 +58,9 @@ def test_probe_library_exports_its_header():
 
 def test_status_strings_and_version(lib):
     from linear_memory_attention_b200 import lard
-    assert [lard.lard_status_string(c) for c in range(5)] == [
+    assert [lard.lard_status_string(c) for c in range(6)] == [
         "LARD_OK", "LARD_ERR_INVALID_ARG", "LARD_ERR_UNSUPPORTED", "LARD_ERR_CUDA",
-        "LARD_ERR_TIMEOUT"]
+        "LARD_ERR_TIMEOUT", "LARD_ERR_TOO_LARGE"]
     assert lard.lard_status_string(99) == "LARD_ERR_UNKNOWN"
     assert lard.lard_version() >= 100
 
