@@ -3,7 +3,9 @@
 
 One step = forward (Phase 1) and backward (Phase 2) of the Q/Q, K/K and V/V
 self-relations of one batch of synthetic RoPE-shaped projections, through
-the C ABI (liblard.so).  Default workload: B=1, H=32, n=32768, d=128, bf16.
+the C ABI (liblard.so): the summed loss and each relation's student gradient
+dL/dX_s (for a self-relation the sum of the two partials, formed in the
+kernel), written as bf16.  Default workload: B=1, H=32, n=32768, d=128, bf16.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lard|reference]
 
@@ -50,9 +52,10 @@ def parse_args():
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: every rank runs its own batch; strong: the ranks split one job's "
                          "(relation, b, h) units and all-reduce the loss")
-    ap.add_argument("--grads", choices=["partials", "dq", "partials-bf16", "dq-bf16"], default="partials",
-                    help="partials: dX_s and dY_s; dq: the fused self-relation gradient dX_s + dY_s; "
-                         "-bf16: the same written as bf16 (fp32 accumulation, rounded once)")
+    ap.add_argument("--grads", choices=["dq-bf16", "dq", "partials", "partials-bf16"], default="dq-bf16",
+                    help="dq: the self-relation gradient dL/dX_s = dX_s + dY_s, fused in the kernel; "
+                         "partials: dX_s and dY_s apart; -bf16: written as bf16 (fp32 accumulation, "
+                         "rounded once), else fp32.  Default dq-bf16: what a bf16 training step consumes")
     ap.add_argument("--no-probe", action="store_true", help="skip the exponential-unit probe")
     return ap.parse_args()
 

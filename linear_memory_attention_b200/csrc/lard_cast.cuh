@@ -21,7 +21,7 @@ struct CastSet {
 
 // Grid-stride over 8-element groups: two 16-byte fp32 loads, one 16-byte bf16
 // store per group.  The loads bypass L1 and are marked as last use.
-__global__ void __launch_bounds__(256) lard_cast_bf16_kernel(const CastSet s) {
+__global__ void __launch_bounds__(256) lard_cast_bf16_kernel(const __grid_constant__ CastSet s) {
     const long long total = s.start8[s.nrel];
     for (long long q = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
          q += static_cast<long long>(gridDim.x) * blockDim.x) {

@@ -238,7 +238,7 @@ struct LossRowsSet {
 
 // loss_bh[bh] = (1/n) sum_i row_kl[bh, i] (LinearARD notes, 关键设计 1: the
 // row-averaged KL), summed in fp64.
-__global__ void __launch_bounds__(256) lard_loss_rows_kernel(const LossRowsSet s) {
+__global__ void __launch_bounds__(256) lard_loss_rows_kernel(const __grid_constant__ LossRowsSet s) {
     int r = 0;
 #pragma unroll
     for (int k = 1; k < kMaxRelations; ++k)
@@ -269,7 +269,7 @@ struct LossSet {
 
 // loss_total = sum over relations and (batch, head) of loss_bh (the relations'
 // losses add with weight 1, LinearARD notes, 损失函数), summed in fp64.
-__global__ void __launch_bounds__(256) lard_loss_total_kernel(const LossSet s, float* loss_total) {
+__global__ void __launch_bounds__(256) lard_loss_total_kernel(const __grid_constant__ LossSet s, float* loss_total) {
     double acc = 0.0;
     for (int r = 0; r < s.nrel; ++r)
         for (int b = threadIdx.x; b < s.BH[r]; b += blockDim.x) acc += s.loss_bh[r][b];

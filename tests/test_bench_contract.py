@@ -37,14 +37,15 @@ def test_reference_arm_line():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("grads", ["partials", "dq"])
+@pytest.mark.parametrize("grads", [None, "partials", "dq"])
 def test_product_arm_line(grads):
+    """The default step (bf16 fused self-relation gradients) and the fp32 forms."""
     import torch
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     K = 4
-    d = _run(["--workload", "n4096", "--steps", str(K), "--warmup", "3", "--cpu-seconds", "1",
-              "--grads", grads], 900)
+    d = _run(["--workload", "n4096", "--steps", str(K), "--warmup", "3", "--cpu-seconds", "1"] +
+             ([] if grads is None else ["--grads", grads]), 900)
     for k in COMMON + ("roofline", "clocks", "gpu_launches", "extra_hbm", "tflops", "kernel_ms"):
         assert k in d, k
     assert d["n_gpus"] == 1 and d["steps"] == K and d["warmup"] == 3 and d["scaling"] == "weak"
@@ -58,10 +59,10 @@ def test_product_arm_line(grads):
     p1 = d["phase1_roofline"]
     assert p1["bound"] == "alu" and p1["measured_ex2_per_clk_per_sm"] > 0 and 0 < p1["frac"] < 1.5
     e = d["e2e"]
-    grads_bytes = (1 if grads == "dq" else 2) * 3 * 32 * 4096 * 128 * 4
+    grads_bytes = {None: 2, "dq": 4, "partials": 8}[grads] * 3 * 32 * 4096 * 128
     assert e["value"] > 0 and e["unit"] == d["unit"] and e["d2h_bytes_per_step"] == grads_bytes + 4
     assert e["h2d_bytes_per_step"] == 6 * 32 * 4096 * 128 * 2  # six bf16 input tensors per step
-    assert d["gpu_launches"] == 4 * K
+    assert d["gpu_launches"] == (5 if grads is None else 4) * K  # + the rounding pass of bf16 outputs
     x = d["extra_hbm"]
     assert x["state_bytes_expected"] == 12 * 3 * 32 * 4096 + 4 * 3 * 32
     # the allocator rounds each of the 4 state buffers of a relation up to its 512-byte granule
