@@ -396,7 +396,16 @@ def run_lard(args):
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     step_tflops = 12 * d * logits_rank * K / (elapsed_ms / 1e3) / 1e12  # per rank
-    traffic, traffic_basis = _profiled_traffic(f"lard_{dom}_tc_kernel<{d}>", w, args.grads)
+    traffic, traffic_basis = _profiled_traffic(f"lard_{dom}_tc_kernel<{d}>", w,
+                                               args.grads if dom == "bwd" else "partials")
+    # Algorithmic DRAM bytes of one launch of the dominant kernel: the distinct input
+    # tensors once (self-relations: X_t and X_s; Y aliases X), plus for Phase 2 the
+    # fp32 gradient accumulators written once (dX_s, and dY_s unless fused), plus for
+    # Phase 1 the 12 bytes of state per row.
+    in_bytes = sum(t.numel() * t.element_size() for xt, xs in host.values() for t in (xt, xs))
+    grad_elems = units_rank * n * d
+    algo_bytes = (in_bytes + grad_elems * 4 * (1 if fused else 2)) if dom == "bwd" else \
+        (in_bytes + 12 * units_rank * n)
     tiles = _tiles(w, units_rank)
     # Cycles per 128 x 128 tile on one SM, from the kernel's time and the median
     # SM clock sampled during the timed region: comparable across clocks (the
@@ -463,7 +472,7 @@ def run_lard(args):
                          "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
                          "peak_kind": f"bf16 dense, sustained ({peak_src})",
                          "frac_of_burst_peak": ach / burst, "traffic": traffic,
-                         "traffic_basis": traffic_basis,
+                         "traffic_basis": traffic_basis, "algorithmic_bytes": algo_bytes,
                          "cycles_per_tile": cyc_bwd if dom == "bwd" else cyc_fwd,
                          "tensor_cycles_per_tile": ideal[dom],
                          "frac_per_clock": (ideal[dom] / (cyc_bwd if dom == "bwd" else cyc_fwd))

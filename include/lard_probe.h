@@ -29,7 +29,9 @@ extern "C" {
  *   kind    0: ex2.approx.ftz.f32 (one exponential per instruction);
  *           1: ex2.approx.f16x2 (two half-precision exponentials per instruction);
  *           2: the FMA-pipe exp2 of the kernels (range reduction and a degree-5
- *              polynomial on packed fp32 pairs).
+ *              polynomial on packed fp32 pairs);
+ *           3: kind 1 between fp32 values (two fp32 packed to half precision,
+ *              one ex2.approx.f16x2, the results widened back to fp32).
  *   blocks  grid size (256 threads per block), >= 1.
  *   iters   chain steps per thread (8 independent chains per thread), >= 1.
  *   ms      out: elapsed time of the kernel (CUDA events on `stream`).

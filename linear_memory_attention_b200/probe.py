@@ -8,7 +8,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblard_probe.so")
 EXPORTS = ("lard_probe_exp_rate",)
-KINDS = {"ex2_f32": 0, "ex2_f16x2": 1, "exp2_fma_pair": 2}
+KINDS = {"ex2_f32": 0, "ex2_f16x2": 1, "exp2_fma_pair": 2, "ex2_f16x2_via_f32": 3}
 
 
 def _load() -> ctypes.CDLL:

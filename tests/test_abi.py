@@ -52,7 +52,7 @@ def test_probe_library_exports_its_header():
         assert hasattr(probe._lib, name)
     # argument errors return before any CUDA call
     ms, ex = ctypes.c_float(), ctypes.c_double()
-    assert probe._lib.lard_probe_exp_rate(5, 1, 1, ctypes.byref(ms), ctypes.byref(ex), None) == 1
+    assert probe._lib.lard_probe_exp_rate(7, 1, 1, ctypes.byref(ms), ctypes.byref(ex), None) == 1
     assert probe._lib.lard_probe_exp_rate(0, 0, 1, ctypes.byref(ms), ctypes.byref(ex), None) == 1
 
 
