@@ -92,3 +92,26 @@ def test_bf16_outputs_refuse_fp32_inputs(lard):
     with pytest.raises(lard.LardError) as e:
         lard.lard_kl_bwd_multi_bf16(rel, w.tau, True, 1.0, ws)
     assert e.value.status == lard.LARD_ERR_UNSUPPORTED
+
+
+def test_bf16_outputs_grouped_noncausal_and_head_dim_64(lard):
+    """No mask with a ragged tail (n = 2000, 16 row blocks), d = 64, three relations
+    with their own head counts, fused and not, in one launch per phase: one
+    whole head per relation against the oracle."""
+    for causal, d in ((False, 128), (True, 64), (False, 64)):
+        pairs, tau = _pairs((("Q", 3), ("K", 1), ("V", 2)), 1, 2000, d, seed=90 + d, causal=causal)
+        for fused in (False, True):
+            outs, _ = lard.relations_kl(pairs, tau, causal, fused_self=fused, grad_dtype="bf16")
+            torch.cuda.synchronize()
+            lard.lard_device_status()
+            for k, ((xt, xs), g) in enumerate(zip(pairs, outs)):
+                h = xt.shape[1] - 1
+                X_t, X_s = f64(xt[0, h]), f64(xs[0, h])
+                o = oracle.relation(X_t, X_t, X_s, X_s, tau, causal)
+                floor = grad_floor(X_s, X_s, tau, 1.0, 2000)
+                what = f"grouped bf16 causal={causal} d={d} fused={fused} relation {k}"
+                if fused:
+                    assert_grad_close(f64(g["dXs"][0, h]), o["dXs"] + o["dYs"], TOL["bf16"]["grad"], what + " dQ", floor)
+                else:
+                    assert_grad_close(f64(g["dXs"][0, h]), o["dXs"], TOL["bf16"]["grad"], what + " dXs", floor)
+                    assert_grad_close(f64(g["dYs"][0, h]), o["dYs"], TOL["bf16"]["grad"], what + " dYs", floor)
