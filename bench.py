@@ -138,9 +138,10 @@ def oracle_sample(w, host, seconds, rank_seed=0):
     orc = oracle.default()
     f64 = {rel: (synth.as_f64(xt[0, 0]), synth.as_f64(xs[0, 0])) for rel, (xt, xs) in host.items()}
     n = w.n
-    probe = min(8, n)
-    t0 = time.perf_counter()
     xt, xs = f64[w.relations[0]]
+    orc.rows(xt, xt, xs, xs, w.tau, w.causal, n - min(8, n), n, want_dY=True)  # threads and pages warm
+    probe = min(32, n)
+    t0 = time.perf_counter()
     orc.rows(xt, xt, xs, xs, w.tau, w.causal, n - probe, n, want_dY=True)
     per_row = (time.perf_counter() - t0) / probe
     R = int(max(1, min(n, seconds / (per_row * len(w.relations)))))
