@@ -115,3 +115,34 @@ def test_bf16_outputs_grouped_noncausal_and_head_dim_64(lard):
                 else:
                     assert_grad_close(f64(g["dXs"][0, h]), o["dXs"], TOL["bf16"]["grad"], what + " dXs", floor)
                     assert_grad_close(f64(g["dYs"][0, h]), o["dYs"], TOL["bf16"]["grad"], what + " dYs", floor)
+
+
+def test_bf16_outputs_cross_relation(lard):
+    """X != Y for teacher and student (a Q K^T map): bf16 dX_s and dY_s from the
+    grouped call, against the oracle, with a ragged n and both masks."""
+    import math
+    from parity_util import random_cross
+    for causal in (True, False):
+        Xt, Yt, Xs, Ys = (t.cuda() for t in random_cross(1, 2, 333, 128, "bf16", seed=77, scale=1.2))
+        tau = 1.0 / math.sqrt(128)
+        f32 = dict(device="cuda", dtype=torch.float32)
+        rel = dict(Xt=Xt, Yt=Yt, Xs=Xs, Ys=Ys, lse_t=torch.empty((1, 2, 333), **f32),
+                   lse_s=torch.empty((1, 2, 333), **f32), row_kl=torch.empty((1, 2, 333), **f32))
+        lard.lard_kl_fwd_multi([rel], tau, causal)
+        out = dict(rel, dXs=torch.empty(Xs.shape, device="cuda", dtype=torch.bfloat16),
+                   dYs=torch.empty(Xs.shape, device="cuda", dtype=torch.bfloat16))
+        out.pop("row_kl")
+        ws = torch.empty((lard.lard_kl_bwd_bf16_workspace_bytes([out]),), device="cuda", dtype=torch.uint8)
+        lard.lard_kl_bwd_multi_bf16([out], tau, causal, 1.0, ws)
+        torch.cuda.synchronize()
+        lard.lard_device_status()
+        for h in range(2):
+            o = oracle.relation(f64(Xt[0, h]), f64(Yt[0, h]), f64(Xs[0, h]), f64(Ys[0, h]), tau, causal)
+            floor = grad_floor(f64(Xs[0, h]), f64(Ys[0, h]), tau, 1.0, 333)
+            what = f"cross bf16 causal={causal} head {h}"
+            assert_grad_close(f64(out["dXs"][0, h]), o["dXs"], TOL["bf16"]["grad"], what + " dXs", floor)
+            assert_grad_close(f64(out["dYs"][0, h]), o["dYs"], TOL["bf16"]["grad"], what + " dYs", floor)
+        # a cross relation has no fused form
+        bad = dict(out, dYs=None)
+        with pytest.raises(lard.LardError):
+            lard.lard_kl_bwd_multi_bf16([bad], tau, causal, 1.0, ws)
