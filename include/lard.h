@@ -35,9 +35,10 @@
  *   - Tensors are row-major [B, H, n, d], contiguous, in device memory of
  *     the GPU that runs the call, base addresses 16-byte aligned.  Inputs
  *     are bf16 (LARD_DTYPE_BF16) or fp32 (LARD_DTYPE_FP32); every output is
- *     fp32, except the gradients of lard_kl_bwd_multi_bf16.  The caller
- *     allocates and owns every buffer (and that call's workspace); the
- *     library allocates no device memory.
+ *     fp32, except the gradients of the two _bf16 Phase-2 calls.  The caller
+ *     allocates and owns every buffer (and the workspace of
+ *     lard_kl_bwd_multi_bf16); the library allocates no device memory (the
+ *     no-allocation variant uses a fixed array that the library holds).
  *   - Work is enqueued asynchronously on `stream` (0 = legacy default
  *     stream); results are valid once the stream reaches that point.
  *   - Argument errors are reported synchronously, before anything is
@@ -47,7 +48,8 @@
  *     lard_device_status() reports as LARD_ERR_TIMEOUT.
  *   - Supported: d in {64, 128} for bf16, d a multiple of 32 up to 256 for
  *     fp32; any n >= 1 (ragged last tile handled); B*H*n*d < 2^40.
- *   - Calls are thread-safe.  Inputs may alias each other (Y = X).
+ *   - Calls are thread-safe (lard_kl_bwd_multi_bf16_noalloc: see its note on
+ *     overlapping calls).  Inputs may alias each other (Y = X).
  */
 #ifndef LARD_H
 #define LARD_H
