@@ -288,11 +288,12 @@ LARD_API const char* lard_status_string(lard_status s);
 LARD_API lard_status lard_device_status(cudaStream_t stream, unsigned int* fault_bits);
 
 /*
- * Failure-detection self-test: enqueues one small kernel whose single wait
- * (an mbarrier that nothing arrives at) runs out after `limit_us`
- * microseconds (1 .. 5e6).  The kernel then sets its bit (0x8000) in the
- * device fault word and returns normally, so that a following
- * lard_device_status() reports LARD_ERR_TIMEOUT with that bit while the
+ * Failure-detection self-test: enqueues one small kernel whose wait (an
+ * mbarrier that nothing arrives at) runs out after `limit_us` microseconds
+ * (1 .. 5e6) and sets its bit (0x8000) in the device fault word; an exit
+ * wait on the same barrier then runs out after as long again and sets the
+ * exit-wait bit (0x100).  The kernel returns normally, so that a following
+ * lard_device_status() reports LARD_ERR_TIMEOUT with both bits while the
  * CUDA context stays usable.  The pages define no counterpart; this checks
  * the bounded waits every kernel of this library relies on.
  */

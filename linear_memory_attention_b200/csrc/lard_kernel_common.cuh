@@ -43,9 +43,10 @@ __device__ __forceinline__ int relation_of_block(const Rel (&rel)[kMaxRelations]
     return r;
 }
 
-// Exercises the bounded wait: one thread waits, with a short limit, on an
-// mbarrier that nothing arrives at; the wait runs out, raises the fault word
-// and the kernel returns normally.
+// Exercises the bounded waits: one thread waits, with a short limit, on an
+// mbarrier that nothing arrives at; the wait runs out and raises its bit in
+// the fault word.  Then the exit wait of a block (drain) runs out on the same
+// barrier and raises the drain bit, and the kernel returns normally.
 __global__ void lard_selftest_timeout_kernel(unsigned long long limit_ns) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
@@ -54,6 +55,7 @@ __global__ void lard_selftest_timeout_kernel(unsigned long long limit_ns) {
         ptx::mbar_init(&bar, 1);
         ptx::fence_mbar_init();
         ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns, &g_lard_fault, kFaultSelfTest);
+        drain(&bar, 0, limit_ns);
     }
 }
 

@@ -22,7 +22,8 @@ def test_timed_out_wait_is_reported_and_context_survives(lard):
     with pytest.raises(lard.LardError) as ei:
         lard.lard_device_status()
     assert ei.value.status == lard.LARD_ERR_TIMEOUT
-    assert ei.value.fault_bits & 0x8000
+    assert ei.value.fault_bits & 0x8000       # the wait inside the loop
+    assert ei.value.fault_bits & 0x100        # the block's exit wait
     assert lard.lard_device_status() == 0  # the word was cleared
     # the context still runs real work correctly
     from linear_memory_attention_b200 import synth
