@@ -169,13 +169,14 @@ lard_status check_common(const void* Xt, const void* Yt, const void* Xs, const v
                          int B, int H, int n, int d, float tau, int causal, long long* BH_out) {
     if (!Xt || !Yt || !Xs || !Ys) return LARD_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || n < 1 || d < 1) return LARD_ERR_INVALID_ARG;
+    if (n > INT_MAX - 127) return LARD_ERR_INVALID_ARG;  // row and tile indices stay in int
     if (!(std::isfinite(tau) && tau > 0.f)) return LARD_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return LARD_ERR_INVALID_ARG;
     if (dtype != LARD_DTYPE_BF16 && dtype != LARD_DTYPE_FP32) return LARD_ERR_UNSUPPORTED;
     if (!d_supported(dtype, d)) return LARD_ERR_UNSUPPORTED;
     const long long BH = static_cast<long long>(B) * H;
     if (BH > INT_MAX / 2 || BH * n > kMaxElems / d) return LARD_ERR_INVALID_ARG;
-    const long long T = (n + 127) / 128;
+    const long long T = (static_cast<long long>(n) + 127) / 128;
     if (BH * T > INT_MAX) return LARD_ERR_INVALID_ARG;
     for (const void* p : {Xt, Yt, Xs, Ys})
         if (!aligned(p, 16)) return LARD_ERR_INVALID_ARG;

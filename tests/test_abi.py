@@ -301,3 +301,12 @@ def test_bf16_workspace_bytes(lib):
 ])
 def test_bwd_multi_bf16_rejects_bad_arguments(lib, specs, outs, kw, code):
     assert bwd_multi_bf16(lib, specs, outs, **kw) == code
+
+
+def test_sizes_beyond_the_limits_are_refused(lib):
+    """B*H*n*d must stay below 2^40 and the grid below 2^31 blocks: refused
+    synchronously, before any CUDA call (the pointers are fake)."""
+    assert fwd(lib, B=1 << 12, H=1 << 12, n=1 << 13, d=128) == 1   # 2^44 elements
+    assert bwd(lib, n=(1 << 31) - 1) == 1                          # row indices past int
+    assert fwd(lib, n=(1 << 31) - 127, B=1, H=1, d=64) == 1         # its last tile's rows past int
+    assert fwd(lib, B=1 << 16, H=1 << 15, n=1) == 1                 # B*H past the 2^30 head limit

@@ -385,3 +385,33 @@ def test_head_dim_64_many_tiles(lard, causal):
     tail, Q/Q and V/V, two heads; whole heads against the oracle."""
     w = synth.custom(1, 2, 3000, 64, "bf16", seed=43, relations=("Q", "V"), causal=causal)
     _run_workload(lard, w, _check_heads(w, {"Q": [(0, 1)], "V": [(0, 0)]}))
+
+
+@pytest.mark.parametrize("tau_scale", [0.1, 3.0], ids=["tau_small", "tau_large"])
+@pytest.mark.parametrize("causal", [1, 0], ids=["causal", "full"])
+def test_other_temperatures(lard, tau_scale, causal):
+    """tau is a parameter: a tenth of 1/sqrt(d) (nearly flat rows) and three times it
+    (sharp rows, logits up to about 35), against the oracle."""
+    w = synth.custom(1, 2, 400, 128, "bf16", seed=31)
+    Xt, Xs = synth.make_relation(w, "K")
+    tau = tau_scale * w.tau
+    o = oracle.relation(f64(Xt), f64(Xt), f64(Xs), f64(Xs), tau, causal)
+    g = gpu_relation(lard, Xt, Xt, Xs, Xs, tau, causal)
+    compare_full(g, o, "bf16", f"tau x{tau_scale} causal={causal}", grad_floor(f64(Xs), f64(Xs), tau, 1.0, 400))
+
+
+def test_large_logits_and_later_maxima(lard):
+    """Cross relation where every row's largest logit (about 70) lies in column 5,
+    far from the diagonal block that each row block processes first: the running
+    maxima rise on a later tile and the online rescaling of the sums is exercised."""
+    B, H, n, d = 1, 2, 700, 128
+    Xt, Yt, Xs, Ys = (t.float() for t in random_cross(B, H, n, d, "bf16", seed=123, scale=1.0))
+    g = torch.Generator().manual_seed(5)
+    v = torch.randn((B, H, 1, d), generator=g)
+    Xt, Xs = Xt + 2 * v, Xs + 2 * v + 0.1 * torch.randn((B, H, 1, d), generator=g)
+    Yt[:, :, 5:6], Ys[:, :, 5:6] = 3 * v, 3 * v
+    Xt, Yt, Xs, Ys = (t.to(torch.bfloat16) for t in (Xt, Yt, Xs, Ys))
+    tau = 1.0 / math.sqrt(d)
+    o = oracle.relation(f64(Xt), f64(Yt), f64(Xs), f64(Ys), tau, True)
+    g = gpu_relation(lard, Xt, Yt, Xs, Ys, tau, True)
+    compare_full(g, o, "bf16", "later maxima", grad_floor(f64(Xs), f64(Ys), tau, 1.0, n))
