@@ -47,7 +47,8 @@
  *     makes the kernel stop early and sets a device-side fault word that
  *     lard_device_status() reports as LARD_ERR_TIMEOUT.
  *   - Supported: d in {64, 128} for bf16, d a multiple of 32 up to 256 for
- *     fp32; any n >= 1 (ragged last tile handled); B*H*n*d < 2^40.
+ *     fp32; any n from 1 to 2^31 - 128 (ragged last tile handled);
+ *     B*H*n*d < 2^40.
  *   - Calls are thread-safe (lard_kl_bwd_multi_bf16_noalloc: see its note on
  *     overlapping calls).  Inputs may alias each other (Y = X).
  */
