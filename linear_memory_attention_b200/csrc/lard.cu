@@ -3,6 +3,7 @@
 // of the relation-KL computation runs in the kernels of the included headers.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <climits>
 #include <cmath>
@@ -56,6 +57,13 @@ struct DeviceGuard {
     ~DeviceGuard() {
         if (prev >= 0) cudaSetDevice(prev);
     }
+};
+
+// NVTX range over one call (a profiler that records NVTX shows each phase's
+// enqueue, and correlates the kernels it launched; without one it costs nothing).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
 };
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -288,6 +296,7 @@ size_t bf16_workspace_bytes(const lard_relation* rel, int nrel, int B, int n, in
 
 lard_status kl_fwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
                    int causal, float* loss_total, cudaStream_t stream) {
+    NvtxRange range("lard Phase 1 (LSE, row KL, losses)");
     if (!rel || nrel < 1 || nrel > lard::kMaxRelations) return LARD_ERR_INVALID_ARG;
     long long BH[lard::kMaxRelations];
     Ranges rg;
@@ -395,6 +404,7 @@ struct Bf16Grads {
 
 lard_status kl_bwd(const lard_relation* rel, int nrel, lard_dtype dtype, int B, int n, int d, float tau,
                    int causal, float grad_scale, cudaStream_t stream, const Bf16Grads* b16 = nullptr) {
+    NvtxRange range(b16 ? "lard Phase 2 (gradients, bf16 outputs)" : "lard Phase 2 (gradients)");
     if (!rel || nrel < 1 || nrel > lard::kMaxRelations) return LARD_ERR_INVALID_ARG;
     if (!std::isfinite(grad_scale)) return LARD_ERR_INVALID_ARG;
     if (b16 && !b16->out) return LARD_ERR_INVALID_ARG;
