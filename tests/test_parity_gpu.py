@@ -415,3 +415,11 @@ def test_large_logits_and_later_maxima(lard):
     o = oracle.relation(f64(Xt), f64(Yt), f64(Xs), f64(Ys), tau, True)
     g = gpu_relation(lard, Xt, Yt, Xs, Ys, tau, True)
     compare_full(g, o, "bf16", "later maxima", grad_floor(f64(Xs), f64(Ys), tau, 1.0, n))
+
+
+def test_head_dim_64_long(lard):
+    """d = 64 at n = 32768 (256 row blocks), two relations of two heads in one grouped
+    launch per phase: one whole head (every row, dY_s on every column) against the
+    oracle, and the properties on every output."""
+    w = synth.custom(1, 2, 32768, 64, "bf16", seed=44, relations=("Q", "V"))
+    _grouped_workload(lard, w, {"V": [(0, 1)]})
