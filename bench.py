@@ -380,6 +380,26 @@ def run_lard(args):
     elapsed_ms = ldist.max_over_ranks(elapsed_ms, device=dev)
     value = ldist.job_rate(logits_job, K, elapsed_ms)
 
+    # A timed region shorter than the sampler's period yields at most one sample,
+    # taken after it, at the idle clock.  The per-clock figures then use the
+    # clock sampled while more untimed steps run for about a second.
+    # (The decision and the step count follow from the max-over-ranks time, so every
+    # rank runs the same steps, and the same collectives in strong scaling.)
+    clk_load = clk
+    if elapsed_ms < 1000.0:
+        per_step = max(elapsed_ms / K, 1e-3)
+        extra = int(min(2000, max(1, 1500.0 / per_step)))
+        sampler = ClockSampler(local)
+        sampler.start()
+        for _ in range(extra):
+            step()
+        torch.cuda.synchronize()
+        clk_load = sampler.stop()
+        clk = dict(clk, sm_mhz_under_load=clk_load.get("sm_mhz"),
+                   note="timed region under a second: sm_mhz from the few samples taken in or "
+                        "right after it; sm_mhz_under_load sampled over further untimed steps "
+                        "(used for the per-clock figures)")
+
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
     if not args.no_e2e and R:
@@ -389,7 +409,7 @@ def run_lard(args):
     # ---------------------------------------------------------------- rooflines
     peaks, peak_src = load_peaks()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    mhz = clk.get("sm_mhz")
+    mhz = clk_load.get("sm_mhz")
     dom, dom_ms = ("bwd", bwd_ms) if sum(bwd_ms) >= sum(fwd_ms) else ("fwd", fwd_ms)
     gemms = 4 if dom == "bwd" else 2
     per_launch_flops = 2 * gemms * d * logits_rank
