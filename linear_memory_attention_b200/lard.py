@@ -16,6 +16,7 @@ Functions keep the C names:
     lard_kl_bwd_multi(relations, tau, causal, grad_scale, stream=None)
     lard_kl_bwd_multi_bf16(relations, tau, causal, grad_scale, workspace, stream=None)
     lard_kl_bwd_bf16_workspace_bytes(relations) -> bytes
+    lard_kl_bwd_multi_bf16_noalloc(relations, tau, causal, grad_scale, stream=None)
     lard_device_status(stream=None) -> fault bits (raises on timeout)
     lard_status_string(code), lard_version()
 Tensors are torch tensors [B, H, n, d] (inputs bf16 or fp32, outputs fp32 except
