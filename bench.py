@@ -184,7 +184,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
         "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": w.name, "B": w.B, "heads": w.heads, "n": w.n,
-                                        "d": w.d, "causal": w.causal},
+                                        "d": w.d, "relations": list(w.relations), "causal": w.causal,
+                                        "gradients": "dX_s and dY_s of the sampled rows, fp64",
+                                        "parallelism": "rank 0 only, host cores"},
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
