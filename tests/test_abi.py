@@ -310,3 +310,18 @@ def test_sizes_beyond_the_limits_are_refused(lib):
     assert bwd(lib, n=(1 << 31) - 1) == 1                          # row indices past int
     assert fwd(lib, n=(1 << 31) - 127, B=1, H=1, d=64) == 1         # its last tile's rows past int
     assert fwd(lib, B=1 << 16, H=1 << 15, n=1) == 1                 # B*H past the 2^30 head limit
+
+
+@pytest.mark.parametrize("module", ["lard.py", "probe.py"])
+def test_binding_without_its_library_fails_loudly(tmp_path, module):
+    """The bindings have no fallback: a copy of a binding module with no built
+    library beside it refuses to import, naming the missing library."""
+    import subprocess
+    import sys
+    src = os.path.join(ROOT, "linear_memory_attention_b200", module)
+    dst = tmp_path / module
+    dst.write_text(open(src).read())
+    out = subprocess.run([sys.executable, "-c", f"import {module[:-3]}"], cwd=tmp_path,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0
+    assert "ImportError" in out.stderr and "is not built" in out.stderr
