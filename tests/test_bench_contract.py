@@ -84,3 +84,13 @@ def test_product_arm_job_split_one_rank():
     assert d["scaling"] == "strong" and d["n_gpus"] == 1 and d["value"] > 0
     assert d["config"]["parallelism"].startswith("units1")
     assert d["extra_hbm"]["rows"] == 2 * (32 + 8 + 8) * 8000
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun only rank 0 runs the reference arm and prints its line."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "n4096", "--steps", "1", "--warmup", "0", "--gpus", "2"],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
